@@ -1,0 +1,202 @@
+// common.cuh -- device helpers shared by the NVFP4 kernels (sm_100a only).
+//
+// Format (sources: "NVFP4 Is a Scaling System, Not Just a 4-Bit Number",
+// "The smallest example"; "MXFP4 和 NVFP4 的区别", "数据格式:极简的 E2M1" and
+// "精度核心:两级分层缩放"; "Melatih model dalam 4 bit", "Anatomi NVFP4"):
+// x = e2m1 * e4m3_block_scale * fp32_global_scale, global = amax / (448 * 6).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library is built for sm_100a only"
+#endif
+
+namespace nvfp4 {
+
+constexpr float kGlobalDiv = 2688.0f;   // 448 (E4M3 max) * 6 (E2M1 max)
+
+// ---------------------------------------------------------------- loads ----
+// Streaming 16-byte load that does not allocate in L1 (each byte is read once).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// bf16 halves of a packed word -> binary32 (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Largest |bf16| of a packed pair accumulated as 16-bit unsigned magnitudes:
+// for finite values the magnitude order equals the order of (bits & 0x7FFF).
+__device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t w) {
+    return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+__device__ __forceinline__ uint32_t absmax2_fold(uint32_t acc) {   // -> binary32 bits of the max
+    uint32_t lo = acc & 0xFFFFu, hi = acc >> 16;
+    return (lo > hi ? lo : hi) << 16;
+}
+
+// ------------------------------------------------------- format conversion --
+// E4M3 (FN) encode of s >= 0: round to nearest even, saturating to 448.
+__device__ __forceinline__ uint32_t e4m3_encode(float s) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(s));
+    return out & 0xFFu;
+}
+// E4M3 -> binary32 (exact, through f16).
+__device__ __forceinline__ float e4m3_decode(uint32_t code) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)code));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// E2M1 encode (nearest even, saturating to +-6, sign kept) of 8 values into
+// 8 nibbles, value 2j in the low nibble of byte j.
+__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4, float v5,
+                                           float v6, float v7) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(out)
+        : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+    return out;
+}
+
+// Eight E2M1 codes (a 32-bit word, code 2j in the low nibble of byte j) ->
+// four f16x2 words (exact); half 0 of word k is element 2k.
+__device__ __forceinline__ void e2m1x8_decode(uint32_t word, uint32_t h[4]) {
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(word));
+}
+
+// -------------------------------------------------------------- Philox ----
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): multipliers 0xD2511F53
+// (word 0) and 0xCD9E8D57 (word 2), Weyl key increments 0x9E3779B9 and
+// 0xBB67AE85 between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    }
+    return c;
+}
+
+// 16 random bits for the 8 output elements 8g .. 8g+7 (element e: word e/2,
+// low half for even e).
+__device__ __forceinline__ uint4 sr_bits8(uint64_t seed, uint64_t g) {
+    return philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), 0u, 0u), (uint32_t)seed,
+                         (uint32_t)(seed >> 32));
+}
+__device__ __forceinline__ uint32_t sr_u16(const uint4& w, int e) {
+    const uint32_t word = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
+    return (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+}
+
+// RHT sign mask ("随机 Hadamard 变换": a random diagonal of signs): bit j set
+// <=> d_j = -1; word 0 of Philox4x32-10 at counter (0, 0, 1, 0), key rht_seed.
+__device__ __forceinline__ uint32_t rht_sign_mask(uint64_t rht_seed) {
+    return philox4x32_10(make_uint4(0u, 0u, 1u, 0u), (uint32_t)rht_seed, (uint32_t)(rht_seed >> 32)).x & 0xFFFFu;
+}
+
+// Stochastic rounding onto the E2M1 grid of one scaled value v (|v| may be
+// +inf): between neighbours lo <= |v| < hi (gap 0.5 below 2, 1 below 4, 2
+// below 6), round up iff u < (|v| - lo) / gap * 65536 (equivalently
+// u < ceil(p * 2^16) for the integer u); |v| >= 6 gives 6.  Returns the
+// signed grid value (exactly representable in E2M1).
+__device__ __forceinline__ float sr_grid(float v, uint32_t u) {
+    const float a = fabsf(v);
+    float q;
+    if (a >= 6.0f) {
+        q = 6.0f;
+    } else {
+        const float gap = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+        const float inv = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
+        const float lo = __fmul_rn(floorf(__fmul_rn(a, inv)), gap);
+        const float frac16 = __fmul_rn(__fsub_rn(a, lo), __fmul_rn(65536.0f, inv));
+        const float uf = __fsub_rn(__uint_as_float(0x4B000000u | u), 8388608.0f);
+        q = uf < frac16 ? __fadd_rn(lo, gap) : lo;
+    }
+    return copysignf(q, v);
+}
+
+// Per-block scale derived from the block amax ("精度核心:两级分层缩放";
+// "Anatomi NVFP4"): s = e4m3(RN(bmax / t)), t = RN(6 s_global) (s = 0 when
+// t == 0); multiplier r = RN(1 / RN(s * s_global)).  r == 0 marks a zero
+// scale (every element encodes a signed zero); r == +inf marks a product that
+// underflowed or a reciprocal that overflowed (nonzero elements saturate).
+struct BlockScale {
+    uint32_t code;
+    float r;
+};
+__device__ __forceinline__ BlockScale block_scale(float bmax, float t, float sg) {
+    const float sf = (t == 0.0f) ? 0.0f : __fdiv_rn(bmax, t);
+    BlockScale b;
+    b.code = e4m3_encode(sf);
+    const float sdec = e4m3_decode(b.code);
+    b.r = (sdec == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sdec, sg));
+    return b;
+}
+
+// Scaled value of one element: RN(x * r); the r == +inf case maps nonzero x to
+// +-6 (saturation) and zero x to a signed zero, as the unrounded products do.
+__device__ __forceinline__ float scaled(float x, float r) {
+    return __fmul_rn(x, r);
+}
+__device__ __forceinline__ float scaled_inf(float x) {
+    return x == 0.0f ? x : copysignf(6.0f, x);
+}
+
+// Offset of scale (row r, block b) in the MMA scale layout (see nvfp4.h).
+__host__ __device__ __forceinline__ int64_t mma_scale_offset(int64_t r, int64_t b, int64_t chunks_k) {
+    return ((r >> 7) * chunks_k + (b >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (b & 3);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    return v;
+}
+
+// Reduce the per-CTA amax partials (binary32 bits of non-negative maxima) to
+// the tensor amax; every thread of the block gets it.
+__device__ __forceinline__ float reduce_partials(const uint32_t* __restrict__ partials, int n) {
+    __shared__ uint32_t s_red[32];
+    uint32_t m = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) m = max(m, __ldg(partials + i));
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t v = lane < (int)(blockDim.x >> 5) ? s_red[lane] : 0u;
+        v = __reduce_max_sync(0xFFFFFFFFu, v);
+        if (lane == 0) s_red[0] = v;
+    }
+    __syncthreads();
+    return __uint_as_float(s_red[0]);
+}
+
+}  // namespace nvfp4

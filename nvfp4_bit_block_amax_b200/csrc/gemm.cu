@@ -1,0 +1,465 @@
+// gemm.cu -- block-scaled NVFP4 GEMM on the sm_100a tensor cores.
+//
+// C = alpha * A . B^T, A [M x K] and B [N x K] as packed E2M1 codes (K-major,
+// "TN"), one UE4M3 scale per 16 elements along K for each row, FP32
+// accumulation in tensor memory, alpha = s_global_A * s_global_B.
+// Sources: "Melatih model dalam 4 bit: pengaman numerik di balik NVFP4",
+// "Presisi sebagai tombol throughput" (the matmuls dominate the step);
+// "NVFP4 Is a Scaling System, Not Just a 4-Bit Number", "Hardware support
+// still needs a full sentence" (native block-scaled matrix operations on
+// Blackwell tensor cores) and "“4-bit” is a payload count" (TN-only GEMM
+// layout, padded/swizzled scale layout).
+//
+// Design (one CTA per SM, persistent over 128 x 256 output tiles, tiles
+// ordered M-fastest so the A panel stays in L2 while B streams):
+//   warp 0      TMA producer: A tile 128 x 256 codes, B tile 256 x 256 codes
+//               (128-byte swizzled), scale chunks by bulk copy; 4 stages.
+//   warp 1      TMEM allocator and MMA issuer: per 64-wide K step, copies
+//               the step's scales smem -> TMEM (tcgen05.cp) and issues
+//               tcgen05.mma kind::mxf4nvf4 block_scale scale_vec::4X with
+//               M = 128, N = 256; commits free smem stages and signal the
+//               accumulator.
+//   warps 2..9  epilogue: TMEM -> registers (128 columns per thread), free
+//               the accumulator for the next tile, scale by alpha, store.
+// Every mbarrier wait is bounded in time: on expiry the kernel raises the
+// device error word, lets in-flight copies and MMAs land, frees TMEM and
+// returns (nvfp4_get_error reports NVFP4_ERR_TIMEOUT).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace nvfp4 {
+
+__device__ unsigned int g_error_word = 0;
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 256;          // elements
+constexpr int BKB = BK / 2;                          // bytes of codes per row per stage
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BKB;                    // 16 KB
+constexpr int B_STAGE = BN * BKB;                    // 32 KB
+constexpr int SFA_STAGE = 4 * 512;                   // 4 K-steps x (128 rows x 4 scales)
+constexpr int SFB_STAGE = 2 * 4 * 512;               // 2 row chunks x 4 K-steps
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
+constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
+constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int NUM_BARS = 2 * STAGES + 3;             // full[], empty[], tmem_full, tmem_empty, drain
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;     // + alignment slack
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_WARPS = 8;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t ACC_COL = 0;
+constexpr uint32_t SF_COL = 256;                     // two buffers of 48 columns
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+
+// ------------------------------------------------------------- PTX wrappers --
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait: false when the limit ran out (the error word and the CTA's
+// abort flag are then set) or another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicExch(&g_error_word, 1u);
+            return false;
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand tile of rows x 128 bytes,
+// 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
+}
+// Descriptor of a 32-row x 16-byte scale chunk (no swizzle, 8-row groups 128
+// bytes apart), the source of tcgen05.cp 32x128b.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(128u >> 4) << 32) |
+           ((uint64_t)1u << 46);
+}
+
+// Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
+// UE4M3 scales, dense K = 64, M = 128, N = 256.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+struct KParams {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const float* a_gs;
+    const float* b_gs;
+    int M, N, K;
+    int chunks_k;
+    int out_bf16;
+    void* c;
+    int64_t ldc;
+    int tiles_m, tiles_n;
+};
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, KParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + OFF_BAR;
+    const uint32_t bar_empty = bar_full + STAGES * 8;
+    const uint32_t bar_tfull = bar_empty + STAGES * 8;
+    const uint32_t bar_tempty = bar_tfull + 8;
+    const uint32_t bar_drain = bar_tempty + 8;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+    const int k_blocks = (p.K + BK - 1) / BK;
+    const int k_steps = p.K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_tfull, 1);
+        mbar_init(bar_tempty, EPI_WARPS);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer ----
+        if (lane == 0) {
+            int s = 0;
+            uint32_t phase = 0;
+            uint32_t issued_parity = 0;   // bit s: parity of the last phase issued on stage s
+            uint32_t issued_any = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+                const int m0 = tm * BM, n0 = tn * BN;
+                const int rc_a = m0 >> 7, rc_b = n0 >> 7;
+                const int rc_b_max = (p.N + 127) >> 7;
+                const int nh = (rc_b + 1 < rc_b_max) ? 2 : 1;
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(bar_empty + 8 * s, phase ^ 1, abort_flag)) { ok = false; break; }
+                    const int nk = min(4, k_steps - kb * 4);
+                    const uint32_t full = bar_full + 8 * s;
+                    mbar_expect_tx(full, (uint32_t)(A_STAGE + B_STAGE + nk * 512 * (1 + nh)));
+                    tma_load_2d(sbase + OFF_A + s * A_STAGE, &map_a, full, kb * BKB, m0);
+                    tma_load_2d(sbase + OFF_B + s * B_STAGE, &map_b, full, kb * BKB, n0);
+                    bulk_load(sbase + OFF_SFA + s * SFA_STAGE,
+                              p.sfa + ((int64_t)rc_a * p.chunks_k + kb * 4) * 512, nk * 512, full);
+                    for (int h = 0; h < nh; ++h)
+                        bulk_load(sbase + OFF_SFB + s * SFB_STAGE + h * 2048,
+                                  p.sfb + ((int64_t)(rc_b + h) * p.chunks_k + kb * 4) * 512, nk * 512, full);
+                    issued_any |= 1u << s;
+                    issued_parity = (issued_parity & ~(1u << s)) | (phase << s);
+                    if (++s == STAGES) { s = 0; phase ^= 1; }
+                }
+            }
+            // let every issued copy land before the CTA can exit
+            for (int st = 0; st < STAGES; ++st)
+                if (issued_any & (1u << st)) {
+                    const uint32_t par = (issued_parity >> st) & 1u;
+                    const unsigned long long t0 = globaltimer();
+                    while (!mbar_try(bar_full + 8 * st, par) && globaltimer() - t0 < kWaitLimitNs) {}
+                }
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------------------------- MMA ----
+        if (lane == 0) {
+            int s = 0;
+            uint32_t phase = 0, acc_phase = 0, kbuf = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                if (!mbar_wait(bar_tempty, acc_phase ^ 1, abort_flag)) break;
+                tc_fence_after();
+                const int n0 = (tile / p.tiles_m) * BN;
+                const int nh = (((n0 >> 7) + 1) < ((p.N + 127) >> 7)) ? 2 : 1;
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(bar_full + 8 * s, phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const int nk = min(4, k_steps - kb * 4);
+                    const uint32_t a_addr = sbase + OFF_A + s * A_STAGE;
+                    const uint32_t b_addr = sbase + OFF_B + s * B_STAGE;
+                    const uint32_t sfa_s = sbase + OFF_SFA + s * SFA_STAGE;
+                    const uint32_t sfb_s = sbase + OFF_SFB + s * SFB_STAGE;
+                    const uint32_t sfa_col = tmem + SF_COL + kbuf * 48;
+                    const uint32_t sfb_col = sfa_col + 16;
+                    for (int j = 0; j < nk; ++j) {
+                        tc_cp_32x128b_x4(sfa_col + 4 * j, desc_sf(sfa_s + j * 512));
+                        for (int h = 0; h < nh; ++h)
+                            tc_cp_32x128b_x4(sfb_col + 8 * j + 4 * h, desc_sf(sfb_s + h * 2048 + j * 512));
+                    }
+                    for (int j = 0; j < nk; ++j) {
+                        tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32), kIdesc,
+                                    sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
+                    }
+                    tc_commit(bar_empty + 8 * s);
+                    kbuf ^= 1;
+                    if (++s == STAGES) { s = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit(bar_tfull);
+                acc_phase ^= 1;
+            }
+            // all MMAs of this CTA complete before TMEM can be freed
+            tc_commit(bar_drain);
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try(bar_drain, 0) && globaltimer() - t0 < kWaitLimitNs) {}
+        }
+    } else {
+        // ------------------------------------------------------ epilogue ----
+        const int q = warp & 3;                 // TMEM lane quarter this warp may access
+        const int half = (warp - 2) >> 2;       // column half of the tile
+        const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+            if (!mbar_wait(bar_tfull, acc_phase, abort_flag)) break;
+            tc_fence_after();
+            const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+            const int row = tm * BM + q * 32 + lane;
+            const int col0 = tn * BN + half * 128;
+            uint32_t v[4][32];
+            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + half * 128;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tc_ld_32x32b_x32(taddr + 32 * i, v[i]);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty);
+            acc_phase ^= 1;
+            if (row < p.M) {
+                if (p.out_bf16) {
+                    __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            const int cc = col0 + 32 * i + 8 * g;
+                            uint32_t w[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __nv_bfloat162 h2 = __floats2bfloat162_rn(
+                                    __fmul_rn(__uint_as_float(v[i][8 * g + 2 * e]), alpha),
+                                    __fmul_rn(__uint_as_float(v[i][8 * g + 2 * e + 1]), alpha));
+                                w[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                            }
+                            if (cc + 8 <= p.N) {
+                                *reinterpret_cast<uint4*>(crow + cc) = make_uint4(w[0], w[1], w[2], w[3]);
+                            } else {
+                                for (int e = 0; e < 8; ++e)
+                                    if (cc + e < p.N) {
+                                        const uint32_t ww = w[e >> 1];
+                                        reinterpret_cast<uint16_t*>(crow)[cc + e] =
+                                            (uint16_t)((e & 1) ? (ww >> 16) : (ww & 0xFFFFu));
+                                    }
+                            }
+                        }
+                    }
+                } else {
+                    float* crow = reinterpret_cast<float*>(p.c) + (int64_t)row * p.ldc;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) {
+                            const int cc = col0 + 32 * i + 4 * g;
+                            const float4 f = make_float4(__fmul_rn(__uint_as_float(v[i][4 * g]), alpha),
+                                                         __fmul_rn(__uint_as_float(v[i][4 * g + 1]), alpha),
+                                                         __fmul_rn(__uint_as_float(v[i][4 * g + 2]), alpha),
+                                                         __fmul_rn(__uint_as_float(v[i][4 * g + 3]), alpha));
+                            if (cc + 4 <= p.N) {
+                                *reinterpret_cast<float4*>(crow + cc) = f;
+                            } else {
+                                const float ff[4] = {f.x, f.y, f.z, f.w};
+                                for (int e = 0; e < 4; ++e)
+                                    if (cc + e < p.N) crow[cc + e] = ff[e];
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
+// ----------------------------------------------------------- host side -----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    });
+    return fn;
+}
+
+bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t k, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)(k / 2), (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(k / 2)};
+    cuuint32_t box[2] = {(cuuint32_t)BKB, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count_cached() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+        cudaFuncSetAttribute(gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    }
+    return cached[dev];
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
+    CUtensorMap ma, mb;
+    if (!make_code_map(&ma, g.a, g.M, g.K, BM) || !make_code_map(&mb, g.b, g.N, g.K, BN))
+        return cudaErrorInvalidValue;
+    KParams p{};
+    p.sfa = g.sfa;
+    p.sfb = g.sfb;
+    p.a_gs = g.a_gs;
+    p.b_gs = g.b_gs;
+    p.M = (int)g.M;
+    p.N = (int)g.N;
+    p.K = (int)g.K;
+    p.chunks_k = (int)mma_chunks_k(g.K);
+    p.out_bf16 = g.out_bf16;
+    p.c = g.c;
+    p.ldc = g.ldc;
+    p.tiles_m = (int)ceil_div(g.M, BM);
+    p.tiles_n = (int)ceil_div(g.N, BN);
+    const int sms = sm_count_cached();
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int grid = tiles < sms ? tiles : sms;
+    gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+    return cudaGetLastError();
+}
+
+unsigned int read_and_clear_error_word(cudaStream_t s, cudaError_t* err) {
+    *err = cudaStreamSynchronize(s);
+    if (*err != cudaSuccess) return 0;
+    unsigned int w = 0;
+    *err = cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w));
+    if (*err != cudaSuccess) return 0;
+    const unsigned int zero = 0;
+    *err = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
+    return w;
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,70 @@
+// internal.h -- host-side launchers shared between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4 {
+
+// Grid of the amax pass: one partial maximum per CTA, reduced by every CTA of
+// the quantize pass that follows on the same stream.
+int amax_grid(int64_t units);
+constexpr int kMaxPartials = 4096;
+
+struct QuantArgs {
+    const uint16_t* x;
+    int64_t rows, cols, ld;       // input [rows x cols], row stride ld (elements)
+    int transpose;                // Q = x (0) or x^T (1)
+    int rht;                      // 16-point RHT along Q rows
+    uint64_t rht_seed;
+    int rounding;                 // 0 RNE, 1 SR
+    uint64_t sr_seed;
+    uint8_t* codes;               // [Qr x Qc/2]
+    uint8_t* scales;              // [Qr x Qc/16] or nullptr
+    uint8_t* scales_mma;          // MMA layout or nullptr
+    float* global_scale;
+    uint32_t* partials;           // workspace
+};
+
+struct Quant2dArgs {
+    const uint16_t* w;
+    int64_t rows, cols, ld;
+    uint8_t* codes_row;
+    uint8_t* codes_col;           // nullable
+    uint8_t* scales;              // nullable
+    uint8_t* scales_mma_row;      // nullable
+    uint8_t* scales_mma_col;      // nullable
+    float* global_scale;
+    uint32_t* partials;
+};
+
+cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches);
+cudaError_t launch_quantize_2d(const Quant2dArgs& a, cudaStream_t s, int* launches);
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int scale_mode, const float* gs,
+                              int64_t rows, int64_t cols, int out_bf16, void* out, cudaStream_t s);
+cudaError_t launch_scales_to_mma(const uint8_t* scales, int scale_mode, int64_t rows, int64_t k,
+                                 uint8_t* scales_mma, cudaStream_t s);
+
+struct GemmArgs {
+    const uint8_t* a;
+    const uint8_t* sfa;
+    const float* a_gs;
+    const uint8_t* b;
+    const uint8_t* sfb;
+    const float* b_gs;
+    int64_t M, N, K;
+    int out_bf16;
+    void* c;
+    int64_t ldc;
+};
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+unsigned int read_and_clear_error_word(cudaStream_t s, cudaError_t* err);
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t mma_chunks_k(int64_t k) { return ceil_div(k / 16, 4); }
+inline size_t mma_scale_bytes(int64_t rows, int64_t k) {
+    return (size_t)(ceil_div(rows, 128) * mma_chunks_k(k) * 512);
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,619 @@
+// quant.cu -- NVFP4 quantizer kernels for sm_100a (HBM-bandwidth bound).
+//
+// Steps (sources: "Melatih model dalam 4 bit: pengaman numerik di balik NVFP4",
+// "Anatomi NVFP4" and "Empat pengaman"; "MXFP4 和 NVFP4 的区别", "精度核心:
+// 两级分层缩放", "随机舍入", "随机 Hadamard 变换", "构造 Hadamard 矩阵的方法";
+// "NVFP4 Is a Scaling System, Not Just a 4-Bit Number", "Why two levels":
+// the global scale comes from the tensor amax before the block maxima):
+//   pass 1 (amax):  A = max |Q| over the tensor (Q rotated when RHT is on);
+//                   one partial maximum per CTA into the caller's workspace.
+//   pass 2 (encode): every CTA folds the partials into A, s_global =
+//                   RN(A / 2688); per 16-block: block amax, E4M3 scale, E2M1
+//                   codes (RNE or stochastic rounding), packed two per byte.
+// All floating-point steps are single IEEE binary32 operations in the order
+// stated in nvfp4.h (this file is built with --fmad=false).
+#include "common.cuh"
+#include "internal.h"
+
+#include <algorithm>
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+// ------------------------------------------------------------ amax (plain) --
+// Tensor amax of a bf16 tensor without rotation: transposing does not change
+// it.  16-byte streaming loads, 16-bit integer magnitude maxima.
+template <bool CONTIG>
+__global__ void __launch_bounds__(kThreads) amax_plain_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                              int64_t cols, int64_t ld,
+                                                              uint32_t* __restrict__ partials) {
+    const int64_t cpr = cols >> 3;
+    const int64_t nvec = rows * cpr;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    auto addr = [&](int64_t i) -> const uint16_t* {
+        if (CONTIG) return x + (i << 3);
+        const int64_t r = i / cpr;
+        return x + r * ld + ((i - r * cpr) << 3);
+    };
+    uint32_t acc = 0;
+    for (; v + (kUnroll - 1) * stride < nvec; v += kUnroll * stride) {
+        uint4 a[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) a[u] = ldg_stream(addr(v + u * stride));
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+            acc = absmax2(absmax2(absmax2(absmax2(acc, a[u].x), a[u].y), a[u].z), a[u].w);
+    }
+    for (; v < nvec; v += stride) {
+        const uint4 a = ldg_stream(addr(v));
+        acc = absmax2(absmax2(absmax2(absmax2(acc, a.x), a.y), a.z), a.w);
+    }
+    __shared__ uint32_t s_red[kThreads / 32];
+    uint32_t m = __reduce_max_sync(0xFFFFFFFFu, absmax2_fold(acc));
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        m = threadIdx.x < (kThreads / 32) ? s_red[threadIdx.x] : 0u;
+        m = __reduce_max_sync(0xFFFFFFFFu, m);
+        if (threadIdx.x == 0) partials[blockIdx.x] = m;
+    }
+}
+
+// Block-level max of non-negative float bits, written as this CTA's partial.
+__device__ __forceinline__ void write_partial(uint32_t m, uint32_t* partials) {
+    __shared__ uint32_t s_red[kThreads / 32];
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        m = threadIdx.x < (kThreads / 32) ? s_red[threadIdx.x] : 0u;
+        m = __reduce_max_sync(0xFFFFFFFFu, m);
+        if (threadIdx.x == 0) partials[blockIdx.x] = m;
+    }
+}
+
+struct Params {
+    const uint16_t* x;
+    int64_t rows, cols, ld;
+    uint64_t rht_seed, sr_seed;
+    uint8_t* codes;
+    uint8_t* scales;
+    uint8_t* scales_mma;
+    int64_t chunks_k;
+    float* global_scale;
+    uint32_t* partials;
+    int n_partials;
+};
+
+// Global scale from the amax partials; block 0 publishes it.
+__device__ __forceinline__ void global_scales(const Params& p, float& sg, float& t) {
+    const float A = reduce_partials(p.partials, p.n_partials);
+    sg = __fdiv_rn(A, kGlobalDiv);
+    t = __fmul_rn(6.0f, sg);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.global_scale = sg;
+}
+
+// 16-point RHT of a chunk split over a lane pair: the even lane holds chunk
+// elements 0..7, the odd lane 8..15.  Sign flips (exact), butterflies
+// h = 1, 2, 4 in registers, h = 8 across the pair, then the factor 1/4.
+__device__ __forceinline__ void rht_pair(float y[8], uint32_t dmask, int lane) {
+    const uint32_t my = (dmask >> ((lane & 1) * 8)) & 0xFFu;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        if ((my >> e) & 1u) y[e] = -y[e];
+#pragma unroll
+    for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            if (i & h) continue;
+            const float a = y[i], b = y[i + h];
+            y[i] = __fadd_rn(a, b);
+            y[i + h] = __fsub_rn(a, b);
+        }
+    }
+    const bool odd = lane & 1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float other = __shfl_xor_sync(0xFFFFFFFFu, y[i], 1);
+        y[i] = odd ? __fsub_rn(other, y[i]) : __fadd_rn(y[i], other);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(y[i], 0.25f);
+}
+
+// ------------------------------------------------- rowwise 1D (Q = x) --------
+// A warp takes consecutive 256-column units of Q rows (lane: 8 columns, a
+// lane pair: one 16-block); 4 units in flight per warp.
+template <bool RHT, bool SR, bool AMAX_ONLY>
+__global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
+    float sg = 0.0f, t = 0.0f;
+    if (!AMAX_ONLY) global_scales(p, sg, t);
+    const uint32_t dmask = RHT ? rht_sign_mask(p.rht_seed) : 0u;
+    const int lane = threadIdx.x & 31;
+    const int64_t hpr = (p.cols + 255) >> 8;
+    const int64_t total = p.rows * hpr;
+    const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+    const int64_t wid = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    const int64_t per = (total + nwarps - 1) / nwarps;
+    int64_t u = wid * per;
+    const int64_t uend = min(total, u + per);
+    const int64_t kb = p.cols >> 4;
+    uint32_t amax_bits = 0;
+    if (u < uend) {
+        int64_t row = u / hpr;
+        int64_t hc = u - row * hpr;
+        for (; u < uend; u += kUnroll) {
+            uint4 v[kUnroll];
+            int64_t rr[kUnroll], cc[kUnroll];
+            bool ok[kUnroll];
+#pragma unroll
+            for (int k = 0; k < kUnroll; ++k) {
+                rr[k] = row;
+                cc[k] = hc * 256 + lane * 8;
+                ok[k] = (u + k < uend) && (cc[k] < p.cols);
+                v[k] = ok[k] ? ldg_stream(p.x + row * p.ld + cc[k]) : make_uint4(0u, 0u, 0u, 0u);
+                if (++hc == hpr) {
+                    hc = 0;
+                    ++row;
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kUnroll; ++k) {
+                if (u + k >= uend) break;  // warp-uniform
+                float y[8] = {bf16_lo(v[k].x), bf16_hi(v[k].x), bf16_lo(v[k].y), bf16_hi(v[k].y),
+                              bf16_lo(v[k].z), bf16_hi(v[k].z), bf16_lo(v[k].w), bf16_hi(v[k].w)};
+                if (RHT) rht_pair(y, dmask, lane);
+                float bmax = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) bmax = fmaxf(bmax, fabsf(y[e]));
+                if (AMAX_ONLY) {
+                    amax_bits = max(amax_bits, __float_as_uint(bmax));
+                    continue;
+                }
+                bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, 1));
+                const BlockScale bs = block_scale(bmax, t, sg);
+                const bool inf_r = isinf(bs.r);
+                float q[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) q[e] = inf_r ? scaled_inf(y[e]) : scaled(y[e], bs.r);
+                if (SR) {
+                    const uint4 rb = sr_bits8(p.sr_seed, (uint64_t)(rr[k] * p.cols + cc[k]) >> 3);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) q[e] = sr_grid(q[e], sr_u16(rb, e));
+                }
+                const uint32_t packed = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+                if (ok[k]) {
+                    *reinterpret_cast<uint32_t*>(p.codes + rr[k] * (p.cols >> 1) + (cc[k] >> 1)) = packed;
+                    if ((lane & 1) == 0) {
+                        const int64_t b = cc[k] >> 4;
+                        if (p.scales) p.scales[rr[k] * kb + b] = (uint8_t)bs.code;
+                        if (p.scales_mma) p.scales_mma[mma_scale_offset(rr[k], b, p.chunks_k)] = (uint8_t)bs.code;
+                    }
+                }
+            }
+        }
+    }
+    if (AMAX_ONLY) write_partial(amax_bits, p.partials);
+}
+
+// ---------------------------------------------- transposed 1D (Q = x^T) -------
+// x is [T x F] (tokens x features); Q = x^T is [F x T] with 16-blocks along
+// tokens.  CTA tile: 128 tokens x 256 features; warp w: tokens 16w..16w+15,
+// lane: 8 features, so a thread holds 8 whole blocks (one per feature) and
+// the RHT runs in registers.  Codes are staged in shared memory and written
+// as 8-byte row segments of Q.
+template <bool RHT, bool SR, bool AMAX_ONLY>
+__global__ void __launch_bounds__(kThreads) cols_kernel(Params p) {
+    __shared__ __align__(16) uint8_t s_codes[256 * 64];
+    float sg = 0.0f, t = 0.0f;
+    if (!AMAX_ONLY) global_scales(p, sg, t);
+    const uint32_t dmask = RHT ? rht_sign_mask(p.rht_seed) : 0u;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t T = p.rows, F = p.cols;
+    const int64_t ntt = (T + 127) >> 7, nft = (F + 255) >> 8;
+    const int64_t ntiles = ntt * nft;
+    const int64_t kb = T >> 4;
+    uint32_t amax_bits = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t tt = tile / nft, ft = tile - tt * nft;
+        const int64_t t0 = tt * 128 + warp * 16;
+        const int64_t f0 = ft * 256 + lane * 8;
+        const bool ok = (t0 < T) && (f0 < F);
+        uint4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            v[i] = ok ? ldg_stream(p.x + (t0 + i) * p.ld + f0) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int jp = 0; jp < 4; ++jp) {
+            float2 y[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                uint32_t w = jp == 0 ? v[i].x : jp == 1 ? v[i].y : jp == 2 ? v[i].z : v[i].w;
+                if (RHT && ((dmask >> i) & 1u)) w ^= 0x80008000u;
+                y[i] = make_float2(bf16_lo(w), bf16_hi(w));
+            }
+            if (RHT) {
+#pragma unroll
+                for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        if (i & h) continue;
+                        const float2 a = y[i], b = y[i + h];
+                        y[i] = __fadd2_rn(a, b);
+                        y[i + h] = __fadd2_rn(a, make_float2(-b.x, -b.y));
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) y[i] = __fmul2_rn(y[i], make_float2(0.25f, 0.25f));
+            }
+            float bm0 = 0.0f, bm1 = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                bm0 = fmaxf(bm0, fabsf(y[i].x));
+                bm1 = fmaxf(bm1, fabsf(y[i].y));
+            }
+            if (AMAX_ONLY) {
+                if (ok) amax_bits = max(amax_bits, __float_as_uint(fmaxf(bm0, bm1)));
+                continue;
+            }
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                const int j = 2 * jp + c;
+                const BlockScale bs = block_scale(c ? bm1 : bm0, t, sg);
+                const bool inf_r = isinf(bs.r);
+                float q[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float yi = c ? y[i].y : y[i].x;
+                    q[i] = inf_r ? scaled_inf(yi) : scaled(yi, bs.r);
+                }
+                if (SR) {
+                    const uint64_t g = (uint64_t)((f0 + j) * T + t0) >> 3;
+                    const uint4 r0 = sr_bits8(p.sr_seed, g);
+                    const uint4 r1 = sr_bits8(p.sr_seed, g + 1);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        q[i] = sr_grid(q[i], sr_u16(r0, i));
+                        q[i + 8] = sr_grid(q[i + 8], sr_u16(r1, i));
+                    }
+                }
+                const uint32_t lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+                const uint32_t hi = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+                const int srow = lane * 8 + j;
+                *reinterpret_cast<uint2*>(s_codes + srow * 64 + ((warp ^ (lane & 7)) * 8)) = make_uint2(lo, hi);
+                if (ok) {
+                    const int64_t f = f0 + j, b = t0 >> 4;
+                    if (p.scales) p.scales[f * kb + b] = (uint8_t)bs.code;
+                    if (p.scales_mma) p.scales_mma[mma_scale_offset(f, b, p.chunks_k)] = (uint8_t)bs.code;
+                }
+            }
+        }
+        if (AMAX_ONLY) continue;
+        __syncthreads();
+        const int64_t fbase = ft * 256, tbyte = tt * 64;
+        const int64_t row_bytes = min((int64_t)64, (T >> 1) - tbyte);
+        for (int k = threadIdx.x; k < 256 * 8; k += kThreads) {
+            const int r = k >> 3, c8 = k & 7;
+            if (fbase + r < F && c8 * 8 < row_bytes) {
+                const uint2 val = *reinterpret_cast<const uint2*>(s_codes + r * 64 + ((c8 ^ ((r >> 3) & 7)) * 8));
+                *reinterpret_cast<uint2*>(p.codes + (fbase + r) * (T >> 1) + tbyte + c8 * 8) = val;
+            }
+        }
+        __syncthreads();
+    }
+    if (AMAX_ONLY) write_partial(amax_bits, p.partials);
+}
+
+// ------------------------------------------------------------ 2D (16x16) ---
+struct Params2d {
+    const uint16_t* w;
+    int64_t rows, cols, ld;
+    uint8_t* codes_row;
+    uint8_t* codes_col;
+    uint8_t* scales;
+    uint8_t* mma_row;
+    uint8_t* mma_col;
+    int64_t chunks_row, chunks_col;
+    float* global_scale;
+    uint32_t* partials;
+    int n_partials;
+};
+
+// CTA tile: 128 rows x 256 columns; warp w: rows 16w..16w+15, lane: 8 columns,
+// a lane pair: one 16x16 tile.  The columnwise codes (of W^T) are the same
+// element codes regrouped along rows, staged in shared memory.
+template <bool COLS>
+__global__ void __launch_bounds__(kThreads) q2d_kernel(Params2d p) {
+    __shared__ __align__(16) uint8_t s_col[COLS ? 256 * 64 : 16];
+    float sg, t;
+    {
+        const float A = reduce_partials(p.partials, p.n_partials);
+        sg = __fdiv_rn(A, kGlobalDiv);
+        t = __fmul_rn(6.0f, sg);
+        if (blockIdx.x == 0 && threadIdx.x == 0) *p.global_scale = sg;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t R = p.rows, C = p.cols;
+    const int64_t ntr = (R + 127) >> 7, ntc = (C + 255) >> 8;
+    const int64_t ntiles = ntr * ntc;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+        const int64_t tr = tile / ntc, tc = tile - tr * ntc;
+        const int64_t r0 = tr * 128 + warp * 16;
+        const int64_t c0 = tc * 256 + lane * 8;
+        const bool ok = (r0 < R) && (c0 < C);
+        uint4 v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = ok ? ldg_stream(p.w + (r0 + i) * p.ld + c0) : make_uint4(0u, 0u, 0u, 0u);
+        uint32_t acc = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc = absmax2(absmax2(absmax2(absmax2(acc, v[i].x), v[i].y), v[i].z), v[i].w);
+        float b = __uint_as_float(absmax2_fold(acc));
+        b = fmaxf(b, __shfl_xor_sync(0xFFFFFFFFu, b, 1));
+        const BlockScale bs = block_scale(b, t, sg);
+        const bool inf_r = isinf(bs.r);
+        auto sc = [&](float x) { return inf_r ? scaled_inf(x) : scaled(x, bs.r); };
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t packed =
+                e2m1x8(sc(bf16_lo(v[i].x)), sc(bf16_hi(v[i].x)), sc(bf16_lo(v[i].y)), sc(bf16_hi(v[i].y)),
+                       sc(bf16_lo(v[i].z)), sc(bf16_hi(v[i].z)), sc(bf16_lo(v[i].w)), sc(bf16_hi(v[i].w)));
+            if (ok) *reinterpret_cast<uint32_t*>(p.codes_row + (r0 + i) * (C >> 1) + (c0 >> 1)) = packed;
+        }
+        if (COLS) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float q[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const uint32_t w = (j >> 1) == 0 ? v[i].x : (j >> 1) == 1 ? v[i].y : (j >> 1) == 2 ? v[i].z : v[i].w;
+                    q[i] = sc((j & 1) ? bf16_hi(w) : bf16_lo(w));
+                }
+                const uint32_t lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+                const uint32_t hi = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+                *reinterpret_cast<uint2*>(s_col + (lane * 8 + j) * 64 + ((warp ^ (lane & 7)) * 8)) = make_uint2(lo, hi);
+            }
+        }
+        if (ok) {
+            const int64_t tb = c0 >> 4, trow = r0 >> 4;
+            if ((lane & 1) == 0) {
+                if (p.scales) p.scales[trow * (C >> 4) + tb] = (uint8_t)bs.code;
+                if (p.mma_row) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) p.mma_row[mma_scale_offset(r0 + i, tb, p.chunks_row)] = (uint8_t)bs.code;
+                }
+            }
+            if (p.mma_col) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) p.mma_col[mma_scale_offset(c0 + j, trow, p.chunks_col)] = (uint8_t)bs.code;
+            }
+        }
+        if (COLS) {
+            __syncthreads();
+            const int64_t cbase = tc * 256, rbyte = tr * 64;
+            const int64_t row_bytes = min((int64_t)64, (R >> 1) - rbyte);
+            for (int k = threadIdx.x; k < 256 * 8; k += kThreads) {
+                const int r = k >> 3, c8 = k & 7;
+                if (cbase + r < C && c8 * 8 < row_bytes) {
+                    const uint2 val = *reinterpret_cast<const uint2*>(s_col + r * 64 + ((c8 ^ ((r >> 3) & 7)) * 8));
+                    *reinterpret_cast<uint2*>(p.codes_col + (cbase + r) * (R >> 1) + rbyte + c8 * 8) = val;
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
+// ------------------------------------------------------------- dequantize ---
+// One thread per 16-block: out = RN(RN(value * s_dec) * s_global).
+__global__ void __launch_bounds__(kThreads) dequant_kernel(const uint8_t* __restrict__ codes,
+                                                          const uint8_t* __restrict__ scales, int mode2d,
+                                                          const float* __restrict__ gs, int64_t rows,
+                                                          int64_t cols, int out_bf16, void* __restrict__ out) {
+    const float sg = __ldg(gs);
+    const int64_t kb = cols >> 4;
+    const int64_t total = rows * kb;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < total;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        const uint2 cw = __ldg(reinterpret_cast<const uint2*>(codes) + u);
+        int64_t si = u;
+        if (mode2d) {
+            const int64_t r = u / kb;
+            si = (r >> 4) * kb + (u - r * kb);
+        }
+        const float s = e4m3_decode(__ldg(scales + si));
+        float o[16];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint32_t h[4];
+            e2m1x8_decode(half ? cw.y : cw.x, h);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 val = __half22float2(*reinterpret_cast<const __half2*>(&h[k]));
+                o[8 * half + 2 * k] = __fmul_rn(__fmul_rn(val.x, s), sg);
+                o[8 * half + 2 * k + 1] = __fmul_rn(__fmul_rn(val.y, s), sg);
+            }
+        }
+        if (out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(out) + u * 16);
+            uint32_t wv[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(o[2 * k], o[2 * k + 1]);
+                wv[k] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+        } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + u * 16);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = make_float4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        }
+    }
+}
+
+// ------------------------------------------------------------ scale layout ---
+__global__ void __launch_bounds__(kThreads) scales_to_mma_kernel(const uint8_t* __restrict__ scales, int mode2d,
+                                                                int64_t rows, int64_t kb, int64_t chunks_k,
+                                                                int64_t total, uint8_t* __restrict__ dst) {
+    for (int64_t d = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; d < total;
+         d += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t chunk = d >> 9, within = d & 511;
+        const int64_t rc = chunk / chunks_k, kc = chunk - rc * chunks_k;
+        const int64_t r = rc * 128 + ((within >> 2) & 3) * 32 + (within >> 4);
+        const int64_t b = kc * 4 + (within & 3);
+        uint8_t val = 0;
+        if (r < rows && b < kb) val = mode2d ? scales[(r >> 4) * kb + b] : scales[r * kb + b];
+        dst[d] = val;
+    }
+}
+
+template <typename K>
+int grid_for(K kernel, int64_t work_items) {
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0);
+    if (per_sm < 1) per_sm = 1;
+    int64_t g = (int64_t)sm_count() * per_sm;
+    if (g > work_items) g = work_items;
+    if (g < 1) g = 1;
+    if (g > kMaxPartials) g = kMaxPartials;
+    return (int)g;
+}
+
+template <bool RHT, bool SR>
+cudaError_t run_rows(Params p, cudaStream_t s, int* launches) {
+    const int64_t units = p.rows * ((p.cols + 255) >> 8);
+    const int64_t warps_needed = (units + kUnroll - 1) / kUnroll;
+    const int g = grid_for(rows_kernel<RHT, SR, false>, (warps_needed + 7) / 8);
+    p.n_partials = g;
+    if (RHT) {
+        rows_kernel<true, false, true><<<g, kThreads, 0, s>>>(p);
+    } else {
+        const bool contig = p.ld == p.cols;
+        if (contig) amax_plain_kernel<true><<<g, kThreads, 0, s>>>(p.x, p.rows, p.cols, p.ld, p.partials);
+        else amax_plain_kernel<false><<<g, kThreads, 0, s>>>(p.x, p.rows, p.cols, p.ld, p.partials);
+    }
+    rows_kernel<RHT, SR, false><<<g, kThreads, 0, s>>>(p);
+    *launches += 2;
+    return cudaGetLastError();
+}
+
+template <bool RHT, bool SR>
+cudaError_t run_cols(Params p, cudaStream_t s, int* launches) {
+    const int64_t tiles = ((p.rows + 127) >> 7) * ((p.cols + 255) >> 8);
+    const int g = grid_for(cols_kernel<RHT, SR, false>, tiles);
+    p.n_partials = g;
+    if (RHT) {
+        cols_kernel<true, false, true><<<g, kThreads, 0, s>>>(p);
+    } else {
+        const bool contig = p.ld == p.cols;
+        if (contig) amax_plain_kernel<true><<<g, kThreads, 0, s>>>(p.x, p.rows, p.cols, p.ld, p.partials);
+        else amax_plain_kernel<false><<<g, kThreads, 0, s>>>(p.x, p.rows, p.cols, p.ld, p.partials);
+    }
+    cols_kernel<RHT, SR, false><<<g, kThreads, 0, s>>>(p);
+    *launches += 2;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int amax_grid(int64_t units) { return (int)std::min<int64_t>(units, kMaxPartials); }
+
+cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches) {
+    Params p{};
+    p.x = a.x;
+    p.rows = a.rows;
+    p.cols = a.cols;
+    p.ld = a.ld;
+    p.rht_seed = a.rht_seed;
+    p.sr_seed = a.sr_seed;
+    p.codes = a.codes;
+    p.scales = a.scales;
+    p.scales_mma = a.scales_mma;
+    p.global_scale = a.global_scale;
+    p.partials = a.partials;
+    const int64_t qr = a.transpose ? a.cols : a.rows;
+    const int64_t qc = a.transpose ? a.rows : a.cols;
+    p.chunks_k = mma_chunks_k(qc);
+    if (a.scales_mma && ((qr % 128) || ((qc / 16) % 4))) {
+        cudaError_t e = cudaMemsetAsync(a.scales_mma, 0, mma_scale_bytes(qr, qc), s);
+        if (e != cudaSuccess) return e;
+    }
+    const bool sr = a.rounding == 1;
+    if (!a.transpose) {
+        if (a.rht) return sr ? run_rows<true, true>(p, s, launches) : run_rows<true, false>(p, s, launches);
+        return sr ? run_rows<false, true>(p, s, launches) : run_rows<false, false>(p, s, launches);
+    }
+    if (a.rht) return sr ? run_cols<true, true>(p, s, launches) : run_cols<true, false>(p, s, launches);
+    return sr ? run_cols<false, true>(p, s, launches) : run_cols<false, false>(p, s, launches);
+}
+
+cudaError_t launch_quantize_2d(const Quant2dArgs& a, cudaStream_t s, int* launches) {
+    Params2d p{};
+    p.w = a.w;
+    p.rows = a.rows;
+    p.cols = a.cols;
+    p.ld = a.ld;
+    p.codes_row = a.codes_row;
+    p.codes_col = a.codes_col;
+    p.scales = a.scales;
+    p.mma_row = a.scales_mma_row;
+    p.mma_col = a.scales_mma_col;
+    p.chunks_row = mma_chunks_k(a.cols);
+    p.chunks_col = mma_chunks_k(a.rows);
+    p.global_scale = a.global_scale;
+    p.partials = a.partials;
+    if (a.scales_mma_row && ((a.rows % 128) || ((a.cols / 16) % 4))) {
+        cudaError_t e = cudaMemsetAsync(a.scales_mma_row, 0, mma_scale_bytes(a.rows, a.cols), s);
+        if (e != cudaSuccess) return e;
+    }
+    if (a.scales_mma_col && ((a.cols % 128) || ((a.rows / 16) % 4))) {
+        cudaError_t e = cudaMemsetAsync(a.scales_mma_col, 0, mma_scale_bytes(a.cols, a.rows), s);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t tiles = ((a.rows + 127) >> 7) * ((a.cols + 255) >> 8);
+    const int g = a.codes_col ? grid_for(q2d_kernel<true>, tiles) : grid_for(q2d_kernel<false>, tiles);
+    p.n_partials = g;
+    if (a.ld == a.cols) amax_plain_kernel<true><<<g, kThreads, 0, s>>>(a.w, a.rows, a.cols, a.ld, a.partials);
+    else amax_plain_kernel<false><<<g, kThreads, 0, s>>>(a.w, a.rows, a.cols, a.ld, a.partials);
+    if (a.codes_col) q2d_kernel<true><<<g, kThreads, 0, s>>>(p);
+    else q2d_kernel<false><<<g, kThreads, 0, s>>>(p);
+    *launches += 2;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int scale_mode, const float* gs,
+                              int64_t rows, int64_t cols, int out_bf16, void* out, cudaStream_t s) {
+    const int64_t total = rows * (cols >> 4);
+    const int g = grid_for(dequant_kernel, (total + kThreads - 1) / kThreads);
+    dequant_kernel<<<g, kThreads, 0, s>>>(codes, scales, scale_mode, gs, rows, cols, out_bf16, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scales_to_mma(const uint8_t* scales, int scale_mode, int64_t rows, int64_t k,
+                                 uint8_t* scales_mma, cudaStream_t s) {
+    const int64_t total = (int64_t)mma_scale_bytes(rows, k);
+    const int g = grid_for(scales_to_mma_kernel, (total + kThreads - 1) / kThreads);
+    scales_to_mma_kernel<<<g, kThreads, 0, s>>>(scales, scale_mode, rows, k >> 4, mma_chunks_k(k), total,
+                                                scales_mma);
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,115 @@
+"""The C-ABI library: loads without a GPU, exports every declared symbol, and
+rejects bad arguments on the host before any launch (no compute here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_bit_block_amax_b200 import build as B
+from nvfp4_bit_block_amax_b200 import nvfp4 as N
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return N.lib()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for name in ("nvfp4_quantize_1d", "nvfp4_quantize_2d", "nvfp4_rht_quantize_sr", "nvfp4_dequantize",
+                 "nvfp4_gemm"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert set(declared_symbols()) <= set(N.EXPORTS) | {"nvfp4_status_string"}
+
+
+def test_version_and_status_strings(L):
+    assert N.nvfp4_version() >= 100
+    for s in range(7):
+        assert N.nvfp4_status_string(s)
+    assert "unknown" in N.nvfp4_status_string(99)
+
+
+def test_sizes(L):
+    assert N.nvfp4_workspace_size(1, 16) >= 4096 * 4
+    assert N.nvfp4_mma_scale_bytes(1, 16) == 512
+    assert N.nvfp4_mma_scale_bytes(128, 256) == 512 * 4
+    assert N.nvfp4_mma_scale_bytes(129, 256) == 512 * 8
+    assert N.nvfp4_mma_scale_bytes(256, 320) == 2 * 5 * 512
+    assert N.nvfp4_mma_scale_bytes(16, 8) == 0
+
+
+FAKE = 1 << 20          # a 16-byte aligned address that is never dereferenced: every call below
+WS = 1 << 14            # fails validation before touching the device
+
+
+def q1d(L, **kw):
+    a = dict(x=FAKE, rows=32, cols=64, ld=64, tr=0, rnd=0, seed=0, codes=FAKE, scales=FAKE, mma=None,
+             gs=FAKE, ws=FAKE, wsb=WS)
+    a.update(kw)
+    return L.nvfp4_quantize_1d(a["x"], a["rows"], a["cols"], a["ld"], a["tr"], a["rnd"], a["seed"], a["codes"],
+                               a["scales"], a["mma"], a["gs"], a["ws"], a["wsb"], None)
+
+
+def test_quantize_1d_validation(L):
+    assert q1d(L, x=None) == 1
+    assert q1d(L, codes=None) == 1
+    assert q1d(L, scales=None, mma=None) == 1
+    assert q1d(L, rows=0) == 1
+    assert q1d(L, ld=32) == 1
+    assert q1d(L, rnd=2) == 1
+    assert q1d(L, tr=3) == 1
+    assert q1d(L, cols=40, ld=40) == 2            # blocks of 16 along the row
+    assert q1d(L, tr=1, rows=40) == 2             # transposed: rows hold the blocks
+    assert q1d(L, x=FAKE + 2) == 3
+    assert q1d(L, ld=68, cols=64) == 3
+    assert q1d(L, ws=None) == 6
+    assert q1d(L, wsb=16) == 6
+
+
+def test_quantize_2d_and_rht_validation(L):
+    assert L.nvfp4_quantize_2d(FAKE, 40, 64, 64, FAKE, None, FAKE, None, None, FAKE, FAKE, WS, None) == 2
+    assert L.nvfp4_quantize_2d(FAKE, 32, 64, 64, None, None, FAKE, None, None, FAKE, FAKE, WS, None) == 1
+    assert L.nvfp4_quantize_2d(FAKE, 32, 64, 64, FAKE + 8, None, FAKE, None, None, FAKE, FAKE, WS, None) == 3
+    assert L.nvfp4_rht_quantize_sr(FAKE, 32, 64, 64, 0, 1, 5, 1, FAKE, FAKE, None, FAKE, FAKE, WS, None) == 1
+    assert L.nvfp4_rht_quantize_sr(FAKE, 30, 64, 64, 1, 1, 1, 1, FAKE, FAKE, None, FAKE, FAKE, WS, None) == 2
+
+
+def test_dequantize_gemm_validation(L):
+    assert L.nvfp4_dequantize(FAKE, FAKE, 0, FAKE, 4, 40, 0, FAKE, None) == 2
+    assert L.nvfp4_dequantize(FAKE, FAKE, 1, FAKE, 8, 32, 0, FAKE, None) == 2
+    assert L.nvfp4_dequantize(FAKE, FAKE, 2, FAKE, 16, 32, 0, FAKE, None) == 1
+    assert L.nvfp4_dequantize(FAKE, FAKE, 0, FAKE, 16, 32, 5, FAKE, None) == 1
+    g = lambda **kw: L.nvfp4_gemm(kw.get("a", FAKE), FAKE, FAKE, FAKE, FAKE, FAKE, kw.get("M", 128),
+                                  kw.get("N", 128), kw.get("K", 256), kw.get("dt", 1), kw.get("c", FAKE),
+                                  kw.get("ldc", 128), None)
+    assert g(a=None) == 1
+    assert g(M=0) == 1
+    assert g(K=96) == 2
+    assert g(ldc=64) == 1
+    assert g(ldc=132) == 3
+    assert g(c=FAKE + 4) == 3
+    assert g(dt=7) == 1
+    assert L.nvfp4_scales_to_mma(FAKE, 1, 20, 64, FAKE, None) == 2
+
+
+def test_missing_library_raises(monkeypatch, tmp_path):
+    monkeypatch.setattr(N, "_lib", None)
+    monkeypatch.setattr(N, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(OSError):
+        N.lib()
