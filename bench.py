@@ -1,0 +1,464 @@
+"""Benchmark of the NVFP4 MLP training-step hot path on B200.
+
+One step = the quantize kernels and the three block-scaled NVFP4 GEMMs of one
+MLP linear layer's training step (tokens 16384, hidden 8192, ffn 28672):
+    X  [16384 x 8192]  bf16 activations  -> 1D RNE codes            (fprop A)
+    W  [28672 x 8192]  bf16 weight       -> 2D RNE codes, rowwise    (fprop B)
+                                            + columnwise W^T codes   (dgrad B)
+    Y  = X . W^T       [16384 x 28672]   bf16                         (fprop)
+    dY [16384 x 28672] bf16 gradient     -> 1D SR codes              (dgrad A)
+    dX = dY . W        [16384 x 8192]    bf16                         (dgrad)
+    dY^T, X^T          16-point RHT (shared signs), dY SR, X RNE     (wgrad A, B)
+    dW = dY^T . X      [28672 x 8192]    bf16                         (wgrad)
+Inputs are seeded synthetic tensors (bf16) resident in HBM; every input
+tensor is larger than the 126 MB L2, so consecutive steps do not hit in L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  Under torchrun each rank runs an independent
+step on its own GPU (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 quantize GB/s (% HBM peak); block-scaled GEMM TFLOPS (% FP4 peak)"
+WORKLOAD = "mlp_step_t16384_h8192_f28672"
+T, H, F = 16384, 8192, 28672
+FP4_OVER_BF16 = 4.0            # nominal dense FP4 / BF16 tensor peak ratio (9 / 2.25 PFLOP/s)
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------- native arm ----
+class Step:
+    """Device buffers of one MLP step and the launch sequence through the C ABI."""
+
+    def __init__(self, torch, N, G, dev):
+        self.torch, self.N = torch, N
+        t, h, f = T, H, F
+        seed, rht_seed, sr_seed = G.seeds("mlp_step")
+        self.rht_seed, self.sr_seed = rht_seed, sr_seed
+        bf = torch.bfloat16
+        u8 = torch.uint8
+        host = {
+            "x": G.activation(t, h, seed),
+            "w": G.weight(f, h, seed + 1),
+            "dy": G.gradient(t, f, seed + 2),
+        }
+        self.host_np = host
+        self.dev = dev
+        mk = lambda a: torch.from_numpy(a.view(np.int16)).view(bf)
+        self.x = mk(host["x"]).to(dev)
+        self.w = mk(host["w"]).to(dev)
+        self.dy = mk(host["dy"]).to(dev)
+        e = lambda *s: torch.empty(*s, dtype=u8, device=dev)
+        mb = N.nvfp4_mma_scale_bytes
+        self.xq = (e(t, h // 2), e(mb(t, h)))                       # fprop A
+        self.wq = (e(f, h // 2), e(mb(f, h)), e(h, f // 2), e(mb(h, f)))   # fprop B, dgrad B
+        self.dyq = (e(t, f // 2), e(mb(t, f)))                      # dgrad A
+        self.dytq = (e(f, t // 2), e(mb(f, t)))                     # wgrad A
+        self.xtq = (e(h, t // 2), e(mb(h, t)))                      # wgrad B
+        self.gs = torch.zeros(8, dtype=torch.float32, device=dev)
+        self.ws = torch.empty(N.nvfp4_workspace_size(0, 0), dtype=u8, device=dev)
+        self.y = torch.empty(t, f, dtype=bf, device=dev)
+        self.dx = torch.empty(t, h, dtype=bf, device=dev)
+        self.dw = torch.empty(f, h, dtype=bf, device=dev)
+        g = self.gs
+        self.gp = [g[i:i + 1] for i in range(5)]
+        # (name, kind, compulsory bytes (quantize: bf16 read + codes + scales written) or flops,
+        #  bytes the two-pass quantizer moves (amax pass re-reads the input), kernels launched)
+        q1 = 2 + 0.5 + 1 / 16
+        q2 = 2 + 0.5 + 0.5 + 2 / 16
+        self.ops = [
+            ("quantize_1d X (rowwise RNE)", "quant", t * h * q1, t * h * (q1 + 2), 2),
+            ("quantize_2d W (row + col codes)", "quant", f * h * q2, f * h * (q2 + 2), 2),
+            ("gemm fprop", "gemm", 2.0 * t * f * h, 0, 1),
+            ("quantize_1d dY (rowwise SR)", "quant", t * f * q1, t * f * (q1 + 2), 2),
+            ("gemm dgrad", "gemm", 2.0 * t * h * f, 0, 1),
+            ("rht_quantize dY^T (SR)", "quant", t * f * q1, t * f * (q1 + 2), 2),
+            ("rht_quantize X^T (RNE)", "quant", t * h * q1, t * h * (q1 + 2), 2),
+            ("gemm wgrad", "gemm", 2.0 * f * h * t, 0, 1),
+        ]
+
+    def launch(self, i, s):
+        N, ws = self.N, self.ws
+        t, h, f = T, H, F
+        ldb = ws.numel()
+        if i == 0:
+            N.nvfp4_quantize_1d(self.x, t, h, h, 0, N.NVFP4_RNE, 0, self.xq[0], None, self.xq[1], self.gp[0], ws, ldb, s)
+        elif i == 1:
+            N.nvfp4_quantize_2d(self.w, f, h, h, self.wq[0], self.wq[2], None, self.wq[1], self.wq[3], self.gp[1], ws,
+                                ldb, s)
+        elif i == 2:
+            N.nvfp4_gemm(self.xq[0], self.xq[1], self.gp[0], self.wq[0], self.wq[1], self.gp[1], t, f, h,
+                         N.NVFP4_OUT_BF16, self.y, f, s)
+        elif i == 3:
+            N.nvfp4_quantize_1d(self.dy, t, f, f, 0, N.NVFP4_SR, self.sr_seed, self.dyq[0], None, self.dyq[1],
+                                self.gp[2], ws, ldb, s)
+        elif i == 4:
+            N.nvfp4_gemm(self.dyq[0], self.dyq[1], self.gp[2], self.wq[2], self.wq[3], self.gp[1], t, h, f,
+                         N.NVFP4_OUT_BF16, self.dx, h, s)
+        elif i == 5:
+            N.nvfp4_rht_quantize_sr(self.dy, t, f, f, 1, self.rht_seed, N.NVFP4_SR, self.sr_seed + 1, self.dytq[0],
+                                    None, self.dytq[1], self.gp[3], ws, ldb, s)
+        elif i == 6:
+            N.nvfp4_rht_quantize_sr(self.x, t, h, h, 1, self.rht_seed, N.NVFP4_RNE, 0, self.xtq[0], None,
+                                    self.xtq[1], self.gp[4], ws, ldb, s)
+        elif i == 7:
+            N.nvfp4_gemm(self.dytq[0], self.dytq[1], self.gp[3], self.xtq[0], self.xtq[1], self.gp[4], f, h, t,
+                         N.NVFP4_OUT_BF16, self.dw, h, s)
+
+    def run(self, stream, events=None):
+        """Enqueue one step on a torch stream (events, if given, bracket each op)."""
+        s = stream.cuda_stream
+        for i in range(len(self.ops)):
+            if events is not None:
+                events[i][0].record(stream)
+            self.launch(i, s)
+            if events is not None:
+                events[i][1].record(stream)
+
+
+def native(args):
+    import torch
+    import torch.distributed as dist
+    from nvfp4_bit_block_amax_b200 import inputs as G
+    from nvfp4_bit_block_amax_b200 import nvfp4 as N
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    N.lib()
+    step = Step(torch, N, G, dev)
+    s = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    with torch.cuda.stream(s):
+        for _ in range(args.warmup):
+            step.run(s)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error(s.cuda_stream) == 0
+
+    ops = step.ops
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ops]
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = N.nvfp4_kernel_launches()
+    wall0 = time.perf_counter()
+    t0.record(s)
+    for k in range(args.steps):
+        step.run(s, ev[k])
+    t1.record(s)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    launches = N.nvfp4_kernel_launches() - launches0
+    barrier()
+    clk = clocks.stop()
+    assert N.nvfp4_get_error(s.cuda_stream) == 0
+    ms_total = t0.elapsed_time(t1)
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    per_op_ms = [statistics.mean(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps))
+                 for i in range(len(ops))]
+    gemm_flops = sum(o[2] for o in ops if o[1] == "gemm")
+    value = gemm_flops * world / (ms_step * 1e-3) / 1e12
+
+    hbm, bf16, bf16_sus, peak_src = peaks()
+    long_region = ms_total > 2000.0
+    fp4_peak = (bf16_sus if long_region else bf16) * FP4_OVER_BF16
+    kernels = []
+    for (name, kind, work, moved, nk), ms in zip(ops, per_op_ms):
+        if kind == "gemm":
+            ach = work / (ms * 1e-3) / 1e12
+            kernels.append({"op": name, "ms": round(ms, 4), "tflops": round(ach, 1),
+                            "frac_fp4_peak": round(ach / fp4_peak, 4)})
+        else:
+            ach = work / (ms * 1e-3) / 1e9
+            mv = moved / (ms * 1e-3) / 1e9
+            kernels.append({"op": name, "ms": round(ms, 4), "gbs_compulsory": round(ach, 1),
+                            "frac_hbm_compulsory": round(ach / hbm, 4), "gbs_moved": round(mv, 1),
+                            "frac_hbm_moved": round(mv / hbm, 4)})
+    gemm_ms = sum(ms for o, ms in zip(ops, per_op_ms) if o[1] == "gemm")
+    quant_ms = sum(ms for o, ms in zip(ops, per_op_ms) if o[1] == "quant")
+    quant_bytes = sum(o[2] for o in ops if o[1] == "quant")
+    quant_moved = sum(o[3] for o in ops if o[1] == "quant")
+    gemm_ach = gemm_flops / (gemm_ms * 1e-3) / 1e12
+    traffic = load_traffic()
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1 x e2m1 (ue4m3 block scales) -> f32 accumulate, bf16 out; quantizers f32 from bf16",
+        "data": "synthetic (seeded PCG64: N(0,1) activations with 0.05% x100 outliers, N(0,0.015^2) weight, "
+                "Laplace(0,1e-3) gradient with 0.1% x1000 outliers)",
+        "config": {"workload": WORKLOAD, "tokens": T, "hidden": H, "ffn": F,
+                   "step": "quantize X(1D RNE), W(2D RNE, row+col), dY(1D SR), RHT dY^T(SR), RHT X^T(RNE); "
+                           "GEMMs fprop, dgrad, wgrad (bf16 out)",
+                   "l2": "every input tensor > 126 MB L2 (no flush needed)", "parallelism": f"replicas x{world}"},
+        "quantize_gbs_compulsory": round(quant_bytes / (quant_ms * 1e-3) / 1e9, 1),
+        "quantize_frac_hbm_compulsory": round(quant_bytes / (quant_ms * 1e-3) / 1e9 / hbm, 4),
+        "quantize_gbs_moved": round(quant_moved / (quant_ms * 1e-3) / 1e9, 1),
+        "quantize_frac_hbm_moved": round(quant_moved / (quant_ms * 1e-3) / 1e9 / hbm, 4),
+        "peaks": {"hbm_gbs": hbm, "fp4_tflops": round(fp4_peak, 1), "source": peak_src},
+        "gemm_tflops": round(gemm_ach, 1),
+        "gemm_frac_fp4_peak": round(gemm_ach / fp4_peak, 4),
+        "kernels": kernels,
+        "roofline": {"bound": "tensor", "achieved": round(gemm_ach, 1), "peak": round(fp4_peak, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_ach / fp4_peak, 4), "traffic": traffic,
+                     "kernel": "gemm_nvf4_kernel (3 GEMMs, mean over launches)",
+                     "peak_source": f"{peak_src} {'sustained' if long_region else 'burst'} bf16 x {FP4_OVER_BF16} "
+                                    "(nominal FP4/BF16 dense ratio)"},
+        "clocks": clk,
+        "gpu_launches": int(launches),
+        "wall_s_timed": round(wall, 3),
+    }
+    if not args.no_e2e:
+        result["e2e"] = e2e(torch, N, step, s, args)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        result["cpu_baseline"] = cpu_baseline(target_s=12.0)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def load_traffic():
+    p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if os.path.exists(p):
+        try:
+            return json.load(open(p)).get("bytes_per_launch")
+        except Exception:
+            return None
+    return None
+
+
+def e2e(torch, N, step, s, args):
+    """The same step through the C ABI with host buffers: pinned host inputs
+    copied in, the three bf16 results copied out, every step."""
+    hx = torch.from_numpy(step.host_np["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hw = torch.from_numpy(step.host_np["w"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    hdy = torch.from_numpy(step.host_np["dy"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    oy = torch.empty(step.y.shape, dtype=torch.bfloat16).pin_memory()
+    odx = torch.empty(step.dx.shape, dtype=torch.bfloat16).pin_memory()
+    odw = torch.empty(step.dw.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * 2 for t in (hx, hw, hdy))
+    d2h = sum(t.numel() * 2 for t in (oy, odx, odw))
+    n = max(3, min(args.steps, 10))
+
+    def one():
+        with torch.cuda.stream(s):
+            step.x.copy_(hx, non_blocking=True)
+            step.w.copy_(hw, non_blocking=True)
+            step.dy.copy_(hdy, non_blocking=True)
+            step.run(s)
+            oy.copy_(step.y, non_blocking=True)
+            odx.copy_(step.dx, non_blocking=True)
+            odw.copy_(step.dw, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(n):
+        one()
+    b.record(s)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / n
+    flops = sum(o[2] for o in step.ops if o[1] == "gemm")
+    return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n}
+
+
+# ------------------------------------------------------------- oracle arm ----
+def oracle_step(t, h, f):
+    """The whole step on a [t x h], [f x h], [t x f] sample, in the CPU oracle:
+    quantize (1D RNE, 2D, 1D SR, RHT SR/RNE transposed), dequantize exactly,
+    float64 GEMMs.  Returns (seconds, flops)."""
+    from nvfp4_bit_block_amax_b200 import inputs as G
+    from oracle import oracle as O
+    seed, rs, ss = G.seeds("mlp_step")
+    x = G.activation(t, h, seed)
+    w = G.weight(f, h, seed + 1)
+    dy = G.gradient(t, f, seed + 2)
+    t0 = time.perf_counter()
+    cx, sx, gx = O.quantize_1d(x)
+    cw, ccw, sw, gw = O.quantize_2d(w)
+    xh = O.dequantize_f64(cx, sx, 0, gx, t, h)
+    wh = O.dequantize_f64(cw, sw, 1, gw, f, h)
+    y = xh @ wh.T
+    cd, sd, gd = O.quantize_1d(dy, rounding=1, sr_seed=ss)
+    dyh = O.dequantize_f64(cd, sd, 0, gd, t, f)
+    wth = O.dequantize_f64(ccw, np.ascontiguousarray(sw.T), 1, gw, h, f)
+    dx = dyh @ wth.T
+    ca, sa, ga = O.quantize_1d(dy, transpose=True, rht=True, rht_seed=rs, rounding=1, sr_seed=ss + 1)
+    cb, sb, gb = O.quantize_1d(x, transpose=True, rht=True, rht_seed=rs, rounding=0)
+    dw = O.dequantize_f64(ca, sa, 0, ga, f, t) @ O.dequantize_f64(cb, sb, 0, gb, h, t).T
+    dt = time.perf_counter() - t0
+    del y, dx, dw
+    return dt, 3 * 2.0 * t * h * f
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+SAMPLE = (512, 1024, 2048)   # tokens, hidden, ffn of the oracle's sample of the step
+
+
+def cpu_baseline(target_s=12.0):
+    t, h, f = SAMPLE
+    secs, flops, n = 0.0, 0.0, 0
+    while secs < target_s and n < 8:
+        dt, fl = oracle_step(t, h, f)
+        secs += dt
+        flops += fl
+        n += 1
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} oracle passes of the step at tokens {t}, hidden {h}, ffn {f} (same recipes); scalar C "
+                      "quantizers on 1 thread, float64 BLAS GEMMs", "seconds": round(secs, 2)}
+
+
+def reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    t, h, f = 256, 512, 1024
+    for _ in range(args.warmup):
+        oracle_step(t, h, f)
+    secs, flops = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_step(t, h, f)
+        secs += dt
+        flops += fl
+    v = flops / secs / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizers, f64 GEMM",
+            "data": "synthetic (same seeded recipes)",
+            "config": {"workload": WORKLOAD, "tokens": T, "hidden": H, "ffn": F, "parallelism": "oracle on host"},
+            "cpu_baseline": {"kind": "oracle", "cores": blas_threads(), "value": round(v, 6), "unit": "TFLOP/s",
+                             "sample": f"each step: the whole step at tokens {t}, hidden {h}, ffn {f}"},
+            "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse()
+    if a.impl == "reference":
+        reference(a)
+    else:
+        native(a)

@@ -12,6 +12,14 @@ from tests.helpers import to_device_bf16
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-3
+WORST = {}
+
+
+def bf16_half_ulp(x):
+    """Half a bf16 unit in the last place at |x| (the store rounding of a bf16 output)."""
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(x, 2.0 ** -126)))
+    return 2.0 ** (e - 8)
 
 
 def quantized_pair(a_bits, b_bits, b_2d=False):
@@ -33,15 +41,22 @@ def quantized_pair(a_bits, b_bits, b_2d=False):
     return a, b, a_hat, b_hat
 
 
-def check(c_gpu, a_hat, b_hat, rows=None):
+def check(c_gpu, a_hat, b_hat, rows=None, bf16_out=False, name=""):
+    """|C - C_ref| <= 2e-3 * S; a bf16 output may in addition differ by the
+    half-ulp rounding of its own store."""
     if rows is not None:
         a_hat = a_hat[rows]
         c_gpu = c_gpu[rows]
     ref, s = O.gemm_reference(a_hat, b_hat)
     err = np.abs(c_gpu.astype(np.float64) - ref)
+    if bf16_out:
+        err = np.maximum(err - bf16_half_ulp(ref), 0.0)
+    ratio = err / np.maximum(s, 1e-300)
+    WORST[name] = float(ratio.max())
+    print(f"[gemm tolerance] {name}: worst |C - C_ref| / S = {ratio.max():.3e}")
     bad = err > TOL * s
-    assert not bad.any(), f"{bad.sum()} elements out of tolerance; worst ratio {(err / np.maximum(s, 1e-300)).max()}"
-    return (err / np.maximum(s, 1e-300)).max()
+    assert not bad.any(), f"{bad.sum()} elements out of tolerance; worst ratio {ratio.max()}"
+    return ratio.max()
 
 
 @pytest.mark.parametrize("out_dtype", [N.NVFP4_OUT_F32, N.NVFP4_OUT_BF16])
@@ -52,7 +67,8 @@ def test_gemm_tiny_linear(out_dtype):
                out_dtype=out_dtype)
     torch.cuda.synchronize()
     assert N.nvfp4_get_error() == 0
-    check(c.float().cpu().numpy(), a_hat, b_hat)
+    check(c.float().cpu().numpy(), a_hat, b_hat, bf16_out=out_dtype == N.NVFP4_OUT_BF16,
+          name=f"tiny_linear out={out_dtype}")
 
 
 @pytest.mark.parametrize("mnk", [(128, 256, 256), (384, 512, 1024), (200, 300, 320), (1, 8, 64),
@@ -67,7 +83,7 @@ def test_gemm_shapes_fp32(mnk):
                out_dtype=N.NVFP4_OUT_F32)
     torch.cuda.synchronize()
     assert N.nvfp4_get_error() == 0
-    check(c.cpu().numpy(), a_hat, b_hat)
+    check(c.cpu().numpy(), a_hat, b_hat, name=f"fp32 {mnk}")
 
 
 def test_gemm_bf16_output_and_padding_untouched():
@@ -80,7 +96,7 @@ def test_gemm_bf16_output_and_padding_untouched():
            out_dtype=N.NVFP4_OUT_BF16, out=full[:, :Nn])
     torch.cuda.synchronize()
     assert (full[:, Nn:] == 7.0).all()
-    check(full[:, :Nn].float().cpu().numpy(), a_hat, b_hat)
+    check(full[:, :Nn].float().cpu().numpy(), a_hat, b_hat, bf16_out=True, name="bf16 ldc-padded")
 
 
 def test_gemm_wgrad_rotation_cancels():
@@ -101,7 +117,7 @@ def test_gemm_wgrad_rotation_cancels():
     a_hat = O.dequantize_f64(ca, sa, 0, ga, F, T)
     b_hat = O.dequantize_f64(cb, sb, 0, gb, H, T)
     cg = c.cpu().numpy()
-    check(cg, a_hat, b_hat)
+    check(cg, a_hat, b_hat, name="wgrad rht")
     exact = G.bf16_bits_to_f32(dy).astype(np.float64).T @ G.bf16_bits_to_f32(x).astype(np.float64)
     scale = np.abs(G.bf16_bits_to_f32(dy)).astype(np.float64).T @ np.abs(G.bf16_bits_to_f32(x)).astype(np.float64)
     assert np.abs(cg - exact).max() <= 0.25 * scale.max()

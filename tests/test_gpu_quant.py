@@ -98,7 +98,7 @@ def test_all_bf16_values_sweep():
         check_1d(x, rounding=rounding, sr_seed=1)
     # the same sweep with a moderate amax, so that mid-range values hit every E2M1 decision
     small = h[np.abs(G.bf16_bits_to_f32(h)) < 64]
-    n = (small.size + 1023) // 1024 * 1024
+    n = (small.size + 16 * 1024 - 1) // (16 * 1024) * (16 * 1024)
     y = np.zeros(n, dtype=np.uint16)
     y[: small.size] = small
     y = y.reshape(-1, 1024)
