@@ -49,6 +49,11 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default=None,
+                    choices=["gemm", "quantize_1d", "quantize_1d_sr", "quantize_2d", "rht_t_sr", "rht_t_rne",
+                             "dequantize"],
+                    help="time one kernel family alone on --shape (profiling mode)")
+    ap.add_argument("--shape", default=None, help="M,N,K for gemm; rows,cols otherwise")
     return ap.parse_args()
 
 
@@ -295,7 +300,7 @@ def native(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "e2m1 x e2m1 (ue4m3 block scales) -> f32 accumulate, bf16 out; quantizers f32 from bf16",
+        "dtype": "e2m1/ue4m3 -> f32",
         "data": "synthetic (seeded PCG64: N(0,1) activations with 0.05% x100 outliers, N(0,0.015^2) weight, "
                 "Laplace(0,1e-3) gradient with 0.1% x1000 outliers)",
         "config": {"workload": WORKLOAD, "tokens": T, "hidden": H, "ffn": F,
@@ -456,9 +461,78 @@ def reference(args):
     print(json.dumps(line), flush=True)
 
 
+def micro(args):
+    """One kernel family alone, for profiling (device-resident random inputs).
+    Prints {op, shape, ms, throughput}; not a bench line."""
+    import torch
+    from nvfp4_bit_block_amax_b200 import nvfp4 as N
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    N.lib()
+    dims = [int(v) for v in args.shape.split(",")]
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    s = torch.cuda.Stream(device=dev)
+    if args.op == "gemm":
+        M, Nn, K = dims
+        a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        b = torch.randint(0, 256, (Nn, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        sa = torch.randint(0x30, 0x40, (N.nvfp4_mma_scale_bytes(M, K),), dtype=torch.uint8, device=dev, generator=g)
+        sb = torch.randint(0x30, 0x40, (N.nvfp4_mma_scale_bytes(Nn, K),), dtype=torch.uint8, device=dev, generator=g)
+        gs = torch.ones(2, dtype=torch.float32, device=dev)
+        c = torch.empty(M, Nn, dtype=torch.bfloat16, device=dev)
+        fn = lambda: N.nvfp4_gemm(a, sa, gs[0:1], b, sb, gs[1:2], M, Nn, K, N.NVFP4_OUT_BF16, c, Nn, s)
+        work, unit = 2.0 * M * Nn * K, "TFLOP/s"
+    else:
+        R, C = dims
+        x = torch.randn(R, C, device=dev, generator=g).to(torch.bfloat16)
+        ws = torch.empty(N.nvfp4_workspace_size(R, C), dtype=torch.uint8, device=dev)
+        gs = torch.empty(1, dtype=torch.float32, device=dev)
+        tr = args.op.startswith("rht_t")
+        qr, qc = (C, R) if tr else (R, C)
+        codes = torch.empty(qr, qc // 2, dtype=torch.uint8, device=dev)
+        smma = torch.empty(N.nvfp4_mma_scale_bytes(qr, qc), dtype=torch.uint8, device=dev)
+        unit = "GB/s"
+        if args.op in ("quantize_1d", "quantize_1d_sr"):
+            rnd = N.NVFP4_SR if args.op.endswith("sr") else N.NVFP4_RNE
+            fn = lambda: N.nvfp4_quantize_1d(x, R, C, C, 0, rnd, 7, codes, None, smma, gs, ws, ws.numel(), s)
+            work = R * C * (2 + 0.5 + 1 / 16)
+        elif args.op == "quantize_2d":
+            cc = torch.empty(C, R // 2, dtype=torch.uint8, device=dev)
+            sm2 = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)
+            fn = lambda: N.nvfp4_quantize_2d(x, R, C, C, codes, cc, None, smma, sm2, gs, ws, ws.numel(), s)
+            work = R * C * (2 + 0.5 + 0.5 + 2 / 16)
+        elif args.op == "dequantize":
+            sc = torch.randint(0x30, 0x40, (R, C // 16), dtype=torch.uint8, device=dev, generator=g)
+            out = torch.empty(R, C, dtype=torch.bfloat16, device=dev)
+            gs.fill_(1.0)
+            fn = lambda: N.nvfp4_dequantize(codes, sc, 0, gs, R, C, N.NVFP4_OUT_BF16, out, s)
+            work = R * C * (0.5 + 1 / 16 + 2)
+        else:
+            rnd = N.NVFP4_SR if args.op.endswith("sr") else N.NVFP4_RNE
+            fn = lambda: N.nvfp4_rht_quantize_sr(x, R, C, C, 1, 5, rnd, 6, codes, None, smma, gs, ws, ws.numel(), s)
+            work = R * C * (2 + 0.5 + 1 / 16)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(args.steps):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error(s.cuda_stream) == 0
+    ms = e0.elapsed_time(e1) / args.steps
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    print(json.dumps({"op": args.op, "shape": dims, "ms": round(ms, 4), "throughput": round(work / (ms * 1e-3) / scale, 1),
+                      "unit": unit, "note": "profiling mode (one op alone), not a bench line"}), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
-    if a.impl == "reference":
+    if a.op:
+        micro(a)
+    elif a.impl == "reference":
         reference(a)
     else:
         native(a)
