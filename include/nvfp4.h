@@ -115,6 +115,33 @@ nvfp4_status nvfp4_quantize_1d(const void* x, int64_t rows, int64_t cols, int64_
                                uint8_t* scales_mma, float* global_scale, void* workspace,
                                size_t ws_bytes, void* stream);
 
+/* nvfp4_quantize_1d for callers that cannot allocate device memory.  The
+ * paper has no counterpart to this entry point.
+ * Who needs it: a process whose device memory is all owned by another
+ * allocator (a framework's caching allocator, or an inference engine that
+ * reserves the whole HBM at start-up), and plug-ins or callbacks that are not
+ * allowed to allocate -- they can hand over inputs and outputs but have no
+ * way to provide a scratch buffer.  This entry point takes the arguments of
+ * nvfp4_quantize_1d minus the workspace and allocates nothing: the tensor-
+ * amax scratch (one partial maximum per CTA of the amax pass) is a static
+ * 4 KiB array inside the library (1024 partials), which every GPU that loads
+ * the library holds until the process exits.
+ *   - The first call on a device looks up that array's device address (once
+ *     per device, with that device current); make this first call before any
+ *     stream capture.
+ *   - A call whose amax pass would need more than 1024 partials (more CTAs
+ *     than a 148-SM B200 launches for this kernel) is refused with
+ *     NVFP4_ERR_WORKSPACE before anything is enqueued.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents; each call's amax pass overwrites every entry its encode pass
+ *     reads, so nothing needs clearing between calls.  Calls that overlap on
+ *     the GPU (other streams, or other host threads on the same device) race
+ *     on the array: serialize them.
+ *   Outputs are bit-identical to nvfp4_quantize_1d's. */
+nvfp4_status nvfp4_quantize_1d_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                                       int rounding, uint64_t sr_seed, uint8_t* codes, uint8_t* scales,
+                                       uint8_t* scales_mma, float* global_scale, void* stream);
+
 /* Random Hadamard transform + quantization of a wgrad operand ["随机 Hadamard
  * 变换" -- an orthogonal rotation with a random sign diagonal applied before
  * quantization, only on the weight-gradient GEMM inputs; "构造 Hadamard 矩阵的

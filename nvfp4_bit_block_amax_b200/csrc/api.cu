@@ -103,6 +103,36 @@ nvfp4_status nvfp4_quantize_1d(const void* x, int64_t rows, int64_t cols, int64_
                             global_scale, workspace, ws_bytes, stream);
 }
 
+nvfp4_status nvfp4_quantize_1d_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                                       int rounding, uint64_t sr_seed, uint8_t* codes, uint8_t* scales,
+                                       uint8_t* scales_mma, float* global_scale, void* stream) {
+    // The argument checks of nvfp4_quantize_1d.  There is no caller workspace
+    // here (the scratch is the library's static array), so the workspace check
+    // is given a placeholder that is only compared, never dereferenced.
+    nvfp4_status st = check_quant_common(x, rows, cols, ld, transpose, rounding, codes, scales, scales_mma,
+                                         global_scale, reinterpret_cast<const void*>(uintptr_t(256)),
+                                         kWorkspaceBytes);
+    if (st != NVFP4_OK) return st;
+    QuantArgs a{};
+    a.x = static_cast<const uint16_t*>(x);
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.transpose = transpose;
+    a.rounding = rounding;
+    a.sr_seed = sr_seed;
+    a.codes = codes;
+    a.scales = scales;
+    a.scales_mma = scales_mma;
+    a.global_scale = global_scale;
+    int n = 0;
+    bool too_big = false;
+    cudaError_t e = launch_quantize_1d_noalloc(a, static_cast<cudaStream_t>(stream), &n, &too_big);
+    if (too_big) return NVFP4_ERR_WORKSPACE;
+    g_launches += n;
+    return from_cuda(e);
+}
+
 nvfp4_status nvfp4_rht_quantize_sr(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
                                    uint64_t rht_seed, int rounding, uint64_t sr_seed, uint8_t* codes,
                                    uint8_t* scales, uint8_t* scales_mma, float* global_scale, void* workspace,

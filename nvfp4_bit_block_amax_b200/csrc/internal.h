@@ -40,6 +40,8 @@ struct Quant2dArgs {
 
 cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches);
 cudaError_t launch_quantize_2d(const Quant2dArgs& a, cudaStream_t s, int* launches);
+cudaError_t launch_quantize_1d_noalloc(const QuantArgs& a, cudaStream_t s, int* launches, bool* too_big);
+int noalloc_capacity();
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int scale_mode, const float* gs,
                               int64_t rows, int64_t cols, int out_bf16, void* out, cudaStream_t s);
 cudaError_t launch_scales_to_mma(const uint8_t* scales, int scale_mode, int64_t rows, int64_t k,

@@ -16,6 +16,7 @@
 #include "internal.h"
 
 #include <algorithm>
+#include <mutex>
 
 namespace nvfp4 {
 
@@ -614,6 +615,71 @@ cudaError_t launch_scales_to_mma(const uint8_t* scales, int scale_mode, int64_t 
     scales_to_mma_kernel<<<g, kThreads, 0, s>>>(scales, scale_mode, rows, k >> 4, mma_chunks_k(k), total,
                                                 scales_mma);
     return cudaGetLastError();
+}
+
+
+// ------------------------------------------------------ no-allocation path ---
+// Scratch for callers that cannot allocate device memory (see
+// nvfp4_quantize_1d_noalloc in nvfp4.h).  The amax pass writes one partial
+// maximum per CTA here and the encode pass reads them back.  The array lives
+// in the library's device image: every GPU that loads the library holds it
+// until the process exits, and all calls on a device share it.
+constexpr int kNoAllocPartials = 1024;   // 4 KiB
+static __device__ __align__(256) uint32_t g_noalloc_partials[kNoAllocPartials];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of the static scratch on the current device, looked up once
+// per device (host code only sees a stand-in symbol, never a device address).
+cudaError_t noalloc_scratch(uint32_t** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_partials);
+        if (e != cudaSuccess) return e;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    *out = static_cast<uint32_t*>(g_noalloc_ptr[dev]);
+    return cudaSuccess;
+}
+}  // namespace
+
+int noalloc_capacity() { return kNoAllocPartials; }
+
+// Same launches as launch_quantize_1d, with the partial maxima in the static
+// scratch.  The CTA count of the amax pass is the one the regular path uses;
+// a configuration that would need more partials than the scratch holds is
+// refused (*too_big = true) before anything is enqueued.
+cudaError_t launch_quantize_1d_noalloc(const QuantArgs& a, cudaStream_t s, int* launches, bool* too_big) {
+    *too_big = false;
+    uint32_t* scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return e;
+    int g;
+    const bool sr = a.rounding == 1;
+    if (!a.transpose) {
+        const int64_t units = a.rows * ((a.cols + 255) >> 8);
+        const int64_t warps_needed = (units + kUnroll - 1) / kUnroll;
+        g = sr ? grid_for(rows_kernel<false, true, false>, (warps_needed + 7) / 8)
+               : grid_for(rows_kernel<false, false, false>, (warps_needed + 7) / 8);
+    } else {
+        const int64_t tiles = ((a.rows + 127) >> 7) * ((a.cols + 255) >> 8);
+        g = sr ? grid_for(cols_kernel<false, true, false>, tiles) : grid_for(cols_kernel<false, false, false>, tiles);
+    }
+    if (g > kNoAllocPartials) {
+        *too_big = true;
+        return cudaSuccess;
+    }
+    QuantArgs b = a;
+    b.rht = 0;
+    b.partials = scratch;
+    return launch_quantize_1d(b, s, launches);
 }
 
 }  // namespace nvfp4

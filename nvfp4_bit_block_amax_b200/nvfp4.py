@@ -29,7 +29,7 @@ NVFP4_OUT_F32, NVFP4_OUT_BF16 = 0, 1
 EXPORTS = (
     "nvfp4_version", "nvfp4_status_string", "nvfp4_workspace_size", "nvfp4_mma_scale_bytes",
     "nvfp4_quantize_1d", "nvfp4_rht_quantize_sr", "nvfp4_quantize_2d", "nvfp4_dequantize", "nvfp4_gemm",
-    "nvfp4_scales_to_mma", "nvfp4_kernel_launches", "nvfp4_get_error",
+    "nvfp4_scales_to_mma", "nvfp4_kernel_launches", "nvfp4_get_error", "nvfp4_quantize_1d_noalloc",
 )
 
 _lib = None
@@ -60,6 +60,8 @@ def lib():
         L.nvfp4_mma_scale_bytes.argtypes = [i64, i64]
         L.nvfp4_quantize_1d.restype = ci
         L.nvfp4_quantize_1d.argtypes = [vp, i64, i64, i64, ci, ci, u64, vp, vp, vp, vp, vp, sz, vp]
+        L.nvfp4_quantize_1d_noalloc.restype = ci
+        L.nvfp4_quantize_1d_noalloc.argtypes = [vp, i64, i64, i64, ci, ci, u64, vp, vp, vp, vp, vp]
         L.nvfp4_rht_quantize_sr.restype = ci
         L.nvfp4_rht_quantize_sr.argtypes = [vp, i64, i64, i64, ci, u64, ci, u64, vp, vp, vp, vp, vp, sz, vp]
         L.nvfp4_quantize_2d.restype = ci
@@ -126,6 +128,15 @@ def nvfp4_quantize_1d(x, rows, cols, ld, transpose, rounding, sr_seed, codes, sc
     _check("nvfp4_quantize_1d", lib().nvfp4_quantize_1d(
         _p(x), rows, cols, ld, transpose, rounding, sr_seed, _p(codes), _p(scales), _p(scales_mma),
         _p(global_scale), _p(workspace), ws_bytes, _stream(stream)))
+
+
+def nvfp4_quantize_1d_noalloc(x, rows, cols, ld, transpose, rounding, sr_seed, codes, scales, scales_mma,
+                              global_scale, stream=None):
+    """nvfp4_quantize_1d without a workspace argument: for callers that cannot
+    allocate device memory, the library uses its own static scratch."""
+    _check("nvfp4_quantize_1d_noalloc", lib().nvfp4_quantize_1d_noalloc(
+        _p(x), rows, cols, ld, transpose, rounding, sr_seed, _p(codes), _p(scales), _p(scales_mma),
+        _p(global_scale), _stream(stream)))
 
 
 def nvfp4_rht_quantize_sr(x, rows, cols, ld, transpose, rht_seed, rounding, sr_seed, codes, scales, scales_mma,
