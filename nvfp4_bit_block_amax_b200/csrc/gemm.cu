@@ -10,17 +10,24 @@
 // Blackwell tensor cores) and "“4-bit” is a payload count" (TN-only GEMM
 // layout, padded/swizzled scale layout).
 //
-// Design (one CTA per SM, persistent over 128 x 256 output tiles, tiles
-// ordered M-fastest so the A panel stays in L2 while B streams):
+// Design (one CTA per SM, persistent over 128 x 256 output tiles; tiles are
+// taken in groups of M-tiles so that the concurrently active A and B panels
+// stay resident in L2):
 //   warp 0      TMA producer: A tile 128 x 256 codes, B tile 256 x 256 codes
 //               (128-byte swizzled), scale chunks by bulk copy; 4 stages.
-//   warp 1      TMEM allocator and MMA issuer: per 64-wide K step, copies
-//               the step's scales smem -> TMEM (tcgen05.cp) and issues
-//               tcgen05.mma kind::mxf4nvf4 block_scale scale_vec::4X with
-//               M = 128, N = 256; commits free smem stages and signal the
-//               accumulator.
-//   warps 2..9  epilogue: TMEM -> registers (128 columns per thread), free
-//               the accumulator for the next tile, scale by alpha, store.
+//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::mxf4nvf4
+//               block_scale scale_vec::4X, M = 128, N = 256, K = 64; commits
+//               free smem stages, scale buffers and signal the accumulator.
+//               Nothing but MMAs goes down its tensor pipe: a scale copy
+//               (tcgen05.cp) issued in the same pipe costs about half an MMA.
+//   warps 2..5  one warp per TMEM lane quarter.  (a) Block scales smem ->
+//               registers -> TMEM (tcgen05.st), up to 4 K-blocks ahead of
+//               the MMAs.  (b) Once the next tile's first K-blocks have
+//               their scales, the epilogue of columns 0..127 of the
+//               finished tile.
+//   warps 6..9  epilogue of columns 128..255.  Epilogue: TMEM -> registers
+//               (128 columns per thread, packed to bf16), free the
+//               accumulator for the next tile, then scale by alpha and store.
 // Every mbarrier wait is bounded in time: on expiry the kernel raises the
 // device error word, lets in-flight copies and MMAs land, frees TMEM and
 // returns (nvfp4_get_error reports NVFP4_ERR_TIMEOUT).
@@ -52,14 +59,16 @@ constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-constexpr int NUM_BARS = 2 * STAGES + 3;             // full[], empty[], tmem_full, tmem_empty, drain
+constexpr int NSF = 4;                               // scale-factor buffers in tensor memory
+constexpr int NUM_BARS = 2 * STAGES + 2 * NSF + 3;   // full, empty, sf_full, sf_empty, tmem_full/empty, drain
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;     // + alignment slack
-constexpr int NUM_THREADS = 320;
-constexpr int EPI_WARPS = 8;
+constexpr int NUM_THREADS = 320;                     // 10 warps (at most 3 per SM sub-partition)
+constexpr int EPI_WARPS = 8;                         // warps 2..5: scales -> TMEM + epilogue columns 0..127;
+                                                     // warps 6..9: epilogue columns 128..255
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SF_COL = 256;                     // two buffers of 48 columns
+constexpr uint32_t SF_COL = 256;                     // NSF buffers of 48 columns (16 SFA + 32 SFB)
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 
 // ------------------------------------------------------------- PTX wrappers --
@@ -122,9 +131,6 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                             uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
     asm volatile(
@@ -144,19 +150,33 @@ __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[3
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+__device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
 
 // Shared-memory matrix descriptor: K-major operand tile of rows x 128 bytes,
 // 128-byte swizzle, 8-row groups 1024 bytes apart.
 __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
     return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(1024u >> 4) << 32) |
            ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
-}
-// Descriptor of a 32-row x 16-byte scale chunk (no swizzle, 8-row groups 128
-// bytes apart), the source of tcgen05.cp 32x128b.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t addr) {
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)(128u >> 4) << 32) |
-           ((uint64_t)1u << 46);
 }
 
 // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
@@ -174,7 +194,102 @@ struct KParams {
     void* c;
     int64_t ldc;
     int tiles_m, tiles_n;
+    int group_m;   // tile rasterization: groups of group_m M-tiles, M fastest inside a group
 };
+
+// Tile t -> (tm, tn).  Tiles are taken in groups of group_m M-tiles; inside a
+// group M runs fastest, then N.  The CTAs working at the same time then share
+// group_m A panels and a few B panels, which stay resident in L2.
+__device__ __forceinline__ void tile_coords(int t, const KParams& p, int& tm, int& tn) {
+    const int per_group = p.group_m * p.tiles_n;
+    const int g = t / per_group;
+    const int r = t - g * per_group;
+    const int first = g * p.group_m;
+    const int gm = min(p.group_m, p.tiles_m - first);
+    tm = first + r % gm;
+    tn = r / gm;
+}
+
+// Epilogue of one column half (128 columns) of a finished tile for the
+// calling warp's TMEM lane quarter: TMEM -> registers (bf16 output: packed
+// pairs, 64 registers), arrive on tmem_empty, then store.  False when the
+// bounded wait for the accumulator ran out.
+__device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int half, int q, int lane, uint32_t tmem,
+                                              float alpha, uint32_t bar_tfull, uint32_t bar_tempty,
+                                              uint32_t& acc_phase, volatile int* abort_flag) {
+    if (!mbar_wait(bar_tfull, acc_phase, abort_flag)) return false;
+    tc_fence_after();
+    int tm, tn;
+    tile_coords(tile, p, tm, tn);
+    const int row = tm * BM + q * 32 + lane;
+    const int col0 = tn * BN + half * 128;
+    const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + half * 128;
+    const int ncols = p.N - col0;   // columns of this half inside C
+    if (p.out_bf16) {
+        uint32_t packed[64];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t v[16];
+            tc_ld_32x32b_x16(taddr + 16 * i, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * e]), alpha),
+                                                                __fmul_rn(__uint_as_float(v[2 * e + 1]), alpha));
+                packed[8 * i + e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_tempty);
+        acc_phase ^= 1;
+        if (row < p.M && ncols > 0) {
+            __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + col0;
+            if (ncols >= 128) {
+#pragma unroll
+                for (int g = 0; g < 16; ++g)
+                    *reinterpret_cast<uint4*>(crow + 8 * g) =
+                        make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+            } else {
+#pragma unroll
+                for (int g = 0; g < 64; ++g) {
+                    if (2 * g + 1 < ncols) reinterpret_cast<uint32_t*>(crow)[g] = packed[g];
+                    else if (2 * g < ncols) reinterpret_cast<uint16_t*>(crow)[2 * g] = (uint16_t)(packed[g] & 0xFFFFu);
+                }
+            }
+        }
+    } else {
+        float* crow = reinterpret_cast<float*>(p.c) + (int64_t)row * p.ldc + col0;
+#pragma unroll 1
+        for (int i = 0; i < 4; ++i) {
+            uint32_t v[32];
+            tc_ld_32x32b_x32(taddr + 32 * i, v);
+            tc_wait_ld();
+            if (row < p.M) {
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const int cc = 32 * i + 4 * g;
+                    const float4 f = make_float4(__fmul_rn(__uint_as_float(v[4 * g]), alpha),
+                                                 __fmul_rn(__uint_as_float(v[4 * g + 1]), alpha),
+                                                 __fmul_rn(__uint_as_float(v[4 * g + 2]), alpha),
+                                                 __fmul_rn(__uint_as_float(v[4 * g + 3]), alpha));
+                    if (cc + 4 <= ncols) {
+                        *reinterpret_cast<float4*>(crow + cc) = f;
+                    } else {
+                        const float ff[4] = {f.x, f.y, f.z, f.w};
+                        for (int e = 0; e < 4; ++e)
+                            if (cc + e < ncols) crow[cc + e] = ff[e];
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_tempty);
+        acc_phase ^= 1;
+    }
+    return true;
+}
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, KParams p) {
@@ -183,7 +298,9 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const uint32_t sbase = smem_u32(smem);
     const uint32_t bar_full = sbase + OFF_BAR;
     const uint32_t bar_empty = bar_full + STAGES * 8;
-    const uint32_t bar_tfull = bar_empty + STAGES * 8;
+    const uint32_t bar_sf_full = bar_empty + STAGES * 8;
+    const uint32_t bar_sf_empty = bar_sf_full + NSF * 8;
+    const uint32_t bar_tfull = bar_sf_empty + NSF * 8;
     const uint32_t bar_tempty = bar_tfull + 8;
     const uint32_t bar_drain = bar_tempty + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
@@ -198,6 +315,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < NSF; ++b) {
+            mbar_init(bar_sf_full + 8 * b, 4);
+            mbar_init(bar_sf_empty + 8 * b, 1);
         }
         mbar_init(bar_tfull, 1);
         mbar_init(bar_tempty, EPI_WARPS);
@@ -225,7 +346,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             uint32_t issued_any = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-                const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+                int tm, tn;
+                tile_coords(tile, p, tm, tn);
                 const int m0 = tm * BM, n0 = tn * BN;
                 const int rc_a = m0 >> 7, rc_b = n0 >> 7;
                 const int rc_b_max = (p.N + 127) >> 7;
@@ -257,37 +379,31 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         }
     } else if (warp == 1) {
         // ----------------------------------------------------------- MMA ----
+        // Only MMAs go down the tensor pipe: the block scales are already in
+        // tensor memory, written by the scale warps.
         if (lane == 0) {
-            int s = 0;
-            uint32_t phase = 0, acc_phase = 0, kbuf = 0;
+            int s = 0, b = 0;
+            uint32_t phase = 0, bphase = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 if (!mbar_wait(bar_tempty, acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
-                const int n0 = (tile / p.tiles_m) * BN;
-                const int nh = (((n0 >> 7) + 1) < ((p.N + 127) >> 7)) ? 2 : 1;
                 for (int kb = 0; kb < k_blocks; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * s, phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait(bar_full + 8 * s, phase, abort_flag) ||
+                        !mbar_wait(bar_sf_full + 8 * b, bphase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const int nk = min(4, k_steps - kb * 4);
                     const uint32_t a_addr = sbase + OFF_A + s * A_STAGE;
                     const uint32_t b_addr = sbase + OFF_B + s * B_STAGE;
-                    const uint32_t sfa_s = sbase + OFF_SFA + s * SFA_STAGE;
-                    const uint32_t sfb_s = sbase + OFF_SFB + s * SFB_STAGE;
-                    const uint32_t sfa_col = tmem + SF_COL + kbuf * 48;
+                    const uint32_t sfa_col = tmem + SF_COL + b * 48;
                     const uint32_t sfb_col = sfa_col + 16;
-                    for (int j = 0; j < nk; ++j) {
-                        tc_cp_32x128b_x4(sfa_col + 4 * j, desc_sf(sfa_s + j * 512));
-                        for (int h = 0; h < nh; ++h)
-                            tc_cp_32x128b_x4(sfb_col + 8 * j + 4 * h, desc_sf(sfb_s + h * 2048 + j * 512));
-                    }
-                    for (int j = 0; j < nk; ++j) {
+                    for (int j = 0; j < nk; ++j)
                         tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32), kIdesc,
                                     sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
-                    }
                     tc_commit(bar_empty + 8 * s);
-                    kbuf ^= 1;
+                    tc_commit(bar_sf_empty + 8 * b);
                     if (++s == STAGES) { s = 0; phase ^= 1; }
+                    if (++b == NSF) { b = 0; bphase ^= 1; }
                 }
                 if (!ok) break;
                 tc_commit(bar_tfull);
@@ -298,78 +414,72 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             const unsigned long long t0 = globaltimer();
             while (!mbar_try(bar_drain, 0) && globaltimer() - t0 < kWaitLimitNs) {}
         }
-    } else {
-        // ------------------------------------------------------ epilogue ----
-        const int q = warp & 3;                 // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;       // column half of the tile
+    } else if (warp < 6) {
+        // ------------------------------- scales -> TMEM, and the epilogue ----
+        // Warp q of this group owns TMEM lanes 32q..32q+31.  Per 64-wide K
+        // step j the MMA reads 4 SFA columns (128 rows; every lane quarter a
+        // copy) and 8 SFB columns (256 rows); lane l of every quarter holds
+        // the 16 bytes at offset 16 l of the step's 512-byte scale chunks.
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
-        uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            if (!mbar_wait(bar_tfull, acc_phase, abort_flag)) break;
-            tc_fence_after();
-            const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-            const int row = tm * BM + q * 32 + lane;
-            const int col0 = tn * BN + half * 128;
-            uint32_t v[4][32];
-            const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + half * 128;
+        int s = 0, b = 0;
+        uint32_t phase = 0, bphase = 0, acc_phase = 0;
+        bool ok = true;
+        int prev_tile = -1;
+        const int lead = min(4, k_blocks);   // K-blocks of the next tile prepared before the epilogue
+
+        auto epilogue = [&](int tile) -> bool {
+            return epilogue_half(p, tile, 0, q, lane, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag);
+        };
+
+        for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int kb = 0; kb < k_blocks; ++kb) {
+                if (!mbar_wait(bar_full + 8 * s, phase, abort_flag) ||
+                    !mbar_wait(bar_sf_empty + 8 * b, bphase ^ 1, abort_flag)) { ok = false; break; }
+                const uint32_t sfa_s = sbase + OFF_SFA + s * SFA_STAGE + 16 * lane;
+                const uint32_t sfb_s = sbase + OFF_SFB + s * SFB_STAGE + 16 * lane;
+                uint32_t ra[16], rb0[16], rb1[16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) tc_ld_32x32b_x32(taddr + 32 * i, v[i]);
-            tc_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tempty);
-            acc_phase ^= 1;
-            if (row < p.M) {
-                if (p.out_bf16) {
-                    __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc;
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 va = lds128(sfa_s + j * 512);
+                    ra[4 * j] = va.x; ra[4 * j + 1] = va.y; ra[4 * j + 2] = va.z; ra[4 * j + 3] = va.w;
+                }
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
+                for (int j = 0; j < 4; ++j) {
 #pragma unroll
-                        for (int g = 0; g < 4; ++g) {
-                            const int cc = col0 + 32 * i + 8 * g;
-                            uint32_t w[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const __nv_bfloat162 h2 = __floats2bfloat162_rn(
-                                    __fmul_rn(__uint_as_float(v[i][8 * g + 2 * e]), alpha),
-                                    __fmul_rn(__uint_as_float(v[i][8 * g + 2 * e + 1]), alpha));
-                                w[e] = *reinterpret_cast<const uint32_t*>(&h2);
-                            }
-                            if (cc + 8 <= p.N) {
-                                *reinterpret_cast<uint4*>(crow + cc) = make_uint4(w[0], w[1], w[2], w[3]);
-                            } else {
-                                for (int e = 0; e < 8; ++e)
-                                    if (cc + e < p.N) {
-                                        const uint32_t ww = w[e >> 1];
-                                        reinterpret_cast<uint16_t*>(crow)[cc + e] =
-                                            (uint16_t)((e & 1) ? (ww >> 16) : (ww & 0xFFFFu));
-                                    }
-                            }
-                        }
-                    }
-                } else {
-                    float* crow = reinterpret_cast<float*>(p.c) + (int64_t)row * p.ldc;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-                        for (int g = 0; g < 8; ++g) {
-                            const int cc = col0 + 32 * i + 4 * g;
-                            const float4 f = make_float4(__fmul_rn(__uint_as_float(v[i][4 * g]), alpha),
-                                                         __fmul_rn(__uint_as_float(v[i][4 * g + 1]), alpha),
-                                                         __fmul_rn(__uint_as_float(v[i][4 * g + 2]), alpha),
-                                                         __fmul_rn(__uint_as_float(v[i][4 * g + 3]), alpha));
-                            if (cc + 4 <= p.N) {
-                                *reinterpret_cast<float4*>(crow + cc) = f;
-                            } else {
-                                const float ff[4] = {f.x, f.y, f.z, f.w};
-                                for (int e = 0; e < 4; ++e)
-                                    if (cc + e < p.N) crow[cc + e] = ff[e];
-                            }
-                        }
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 vb = lds128(sfb_s + h * 2048 + j * 512);
+                        uint32_t* rb = j < 2 ? rb0 : rb1;
+                        const int o = 8 * (j & 1) + 4 * h;
+                        rb[o] = vb.x; rb[o + 1] = vb.y; rb[o + 2] = vb.z; rb[o + 3] = vb.w;
                     }
                 }
+                const uint32_t col = tmem + lane_base + SF_COL + b * 48;
+                tc_st_32x32b_x16(col, ra);
+                tc_st_32x32b_x16(col + 16, rb0);
+                tc_st_32x32b_x16(col + 32, rb1);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_sf_full + 8 * b);
+                if (++s == STAGES) { s = 0; phase ^= 1; }
+                if (++b == NSF) { b = 0; bphase ^= 1; }
+                if (kb == lead - 1 && prev_tile >= 0) {
+                    if (!epilogue(prev_tile)) { ok = false; break; }
+                    prev_tile = -1;
+                }
             }
+            if (ok) prev_tile = tile;
         }
+        if (ok && prev_tile >= 0) epilogue(prev_tile);
+    } else {
+        // ---------------------------------------- epilogue, columns 128..255 ----
+        const int q = warp & 3;
+        const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x)
+            if (!epilogue_half(p, tile, 1, q, lane, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag)) break;
     }
 
     tc_fence_before();
@@ -444,6 +554,12 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     p.ldc = g.ldc;
     p.tiles_m = (int)ceil_div(g.M, BM);
     p.tiles_n = (int)ceil_div(g.N, BN);
+    // group as many A panels (128 rows x K/2 bytes each) as fit in ~24 MB of L2
+    const int64_t panel = (int64_t)BM * (g.K / 2);
+    int64_t gm = (24ll << 20) / (panel > 0 ? panel : 1);
+    if (gm < 1) gm = 1;
+    if (gm > p.tiles_m) gm = p.tiles_m;
+    p.group_m = (int)gm;
     const int sms = sm_count_cached();
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < sms ? tiles : sms;

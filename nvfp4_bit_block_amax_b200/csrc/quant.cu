@@ -112,103 +112,172 @@ __device__ __forceinline__ void global_scales(const Params& p, float& sg, float&
     if (blockIdx.x == 0 && threadIdx.x == 0) *p.global_scale = sg;
 }
 
-// 16-point RHT of a chunk split over a lane pair: the even lane holds chunk
-// elements 0..7, the odd lane 8..15.  Sign flips (exact), butterflies
-// h = 1, 2, 4 in registers, h = 8 across the pair, then the factor 1/4.
-__device__ __forceinline__ void rht_pair(float y[8], uint32_t dmask, int lane) {
-    const uint32_t my = (dmask >> ((lane & 1) * 8)) & 0xFFu;
+// 32-byte load of 16 bf16 values (one block).  A single 256-bit load when the
+// address is 32-byte aligned, else two 16-byte loads.
+__device__ __forceinline__ void load_block(const uint16_t* p, bool a32, uint32_t w[8]) {
+    if (a32) {
+        asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+                       "=r"(w[7])
+                     : "l"(p));
+    } else {
+        const uint4 a = ldg_stream(p), b = ldg_stream(p + 8);
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    }
+}
+
+// 16-point RHT of one chunk held by one thread: signs (exact), butterflies
+// h = 1, 2, 4, 8 (pairs of independent butterflies packed into f32x2 adds),
+// then the factor 1/4.
+__device__ __forceinline__ void rht16_regs(float y[16]) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-        if ((my >> e) & 1u) y[e] = -y[e];
+    for (int h = 1; h < 16; h <<= 1) {
+        int idx[8];
+        int n = 0;
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1) {
+        for (int i = 0; i < 16; ++i)
+            if (!(i & h)) idx[n++] = i;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            if (i & h) continue;
-            const float a = y[i], b = y[i + h];
-            y[i] = __fadd_rn(a, b);
-            y[i + h] = __fsub_rn(a, b);
+        for (int k = 0; k < 8; k += 2) {
+            const int i0 = idx[k], i1 = idx[k + 1];
+            const float2 a = make_float2(y[i0], y[i1]);
+            const float2 b = make_float2(y[i0 + h], y[i1 + h]);
+            const float2 sum = __fadd2_rn(a, b);
+            const float2 dif = __fadd2_rn(a, make_float2(-b.x, -b.y));
+            y[i0] = sum.x;
+            y[i1] = sum.y;
+            y[i0 + h] = dif.x;
+            y[i1 + h] = dif.y;
         }
     }
-    const bool odd = lane & 1;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float other = __shfl_xor_sync(0xFFFFFFFFu, y[i], 1);
-        y[i] = odd ? __fsub_rn(other, y[i]) : __fadd_rn(y[i], other);
+    for (int i = 0; i < 16; i += 2) {
+        const float2 v = __fmul2_rn(make_float2(y[i], y[i + 1]), make_float2(0.25f, 0.25f));
+        y[i] = v.x;
+        y[i + 1] = v.y;
     }
+}
+
+// Encode one 16-block held by one thread: codes for elements 0..7 (lo) and
+// 8..15 (hi).  SR draws its bits for output elements 8g .. 8g+15.
+template <bool SR>
+__device__ __forceinline__ void encode16(const float y[16], const BlockScale& bs, uint64_t sr_seed, uint64_t g,
+                                         uint32_t& lo, uint32_t& hi) {
+    float q[16];
+    if (!isinf(bs.r)) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(y[i], 0.25f);
+        for (int i = 0; i < 16; i += 2) {
+            const float2 v = __fmul2_rn(make_float2(y[i], y[i + 1]), make_float2(bs.r, bs.r));
+            q[i] = v.x;
+            q[i + 1] = v.y;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) q[i] = scaled_inf(y[i]);
+    }
+    if (SR) {
+        const uint4 r0 = sr_bits8(sr_seed, g);
+        const uint4 r1 = sr_bits8(sr_seed, g + 1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            q[i] = sr_grid(q[i], sr_u16(r0, i));
+            q[i + 8] = sr_grid(q[i + 8], sr_u16(r1, i));
+        }
+    }
+    lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
+    hi = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
 }
 
 // ------------------------------------------------- rowwise 1D (Q = x) --------
-// A warp takes consecutive 256-column units of Q rows (lane: 8 columns, a
-// lane pair: one 16-block); 4 units in flight per warp.
+// One thread per 16-block: a warp takes 512 consecutive columns of a Q row
+// (32 blocks) per unit, consecutive units per warp, 2 units in flight.
 template <bool RHT, bool SR, bool AMAX_ONLY>
 __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
     float sg = 0.0f, t = 0.0f;
     if (!AMAX_ONLY) global_scales(p, sg, t);
-    const uint32_t dmask = RHT ? rht_sign_mask(p.rht_seed) : 0u;
+    uint32_t sw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (RHT) {
+        const uint32_t d = rht_sign_mask(p.rht_seed);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            sw[k] = (((d >> (2 * k)) & 1u) ? 0x8000u : 0u) | (((d >> (2 * k + 1)) & 1u) ? 0x80000000u : 0u);
+    }
     const int lane = threadIdx.x & 31;
-    const int64_t hpr = (p.cols + 255) >> 8;
-    const int64_t total = p.rows * hpr;
+    const int64_t upr = (p.cols + 511) >> 9;
+    const int64_t total = p.rows * upr;
     const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
     const int64_t wid = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
     const int64_t per = (total + nwarps - 1) / nwarps;
     int64_t u = wid * per;
     const int64_t uend = min(total, u + per);
     const int64_t kb = p.cols >> 4;
+    const bool a32 = ((reinterpret_cast<uintptr_t>(p.x) & 31u) == 0) && ((p.ld & 15) == 0);
     uint32_t amax_bits = 0;
+    constexpr int U = 2;
     if (u < uend) {
-        int64_t row = u / hpr;
-        int64_t hc = u - row * hpr;
-        for (; u < uend; u += kUnroll) {
-            uint4 v[kUnroll];
-            int64_t rr[kUnroll], cc[kUnroll];
-            bool ok[kUnroll];
+        int64_t row = u / upr;
+        int64_t uc = u - row * upr;
+        for (; u < uend; u += U) {
+            uint32_t w[U][8];
+            int64_t rr[U], cc[U];
+            bool ok[U];
 #pragma unroll
-            for (int k = 0; k < kUnroll; ++k) {
+            for (int k = 0; k < U; ++k) {
                 rr[k] = row;
-                cc[k] = hc * 256 + lane * 8;
+                cc[k] = uc * 512 + lane * 16;
                 ok[k] = (u + k < uend) && (cc[k] < p.cols);
-                v[k] = ok[k] ? ldg_stream(p.x + row * p.ld + cc[k]) : make_uint4(0u, 0u, 0u, 0u);
-                if (++hc == hpr) {
-                    hc = 0;
+                if (ok[k]) {
+                    load_block(p.x + row * p.ld + cc[k], a32, w[k]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) w[k][j] = 0u;
+                }
+                if (++uc == upr) {
+                    uc = 0;
                     ++row;
                 }
             }
 #pragma unroll
-            for (int k = 0; k < kUnroll; ++k) {
-                if (u + k >= uend) break;  // warp-uniform
-                float y[8] = {bf16_lo(v[k].x), bf16_hi(v[k].x), bf16_lo(v[k].y), bf16_hi(v[k].y),
-                              bf16_lo(v[k].z), bf16_hi(v[k].z), bf16_lo(v[k].w), bf16_hi(v[k].w)};
-                if (RHT) rht_pair(y, dmask, lane);
-                float bmax = 0.0f;
+            for (int k = 0; k < U; ++k) {
+                float y[16];
+                float bmax;
+                if (RHT) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) bmax = fmaxf(bmax, fabsf(y[e]));
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t ww = w[k][j] ^ sw[j];
+                        y[2 * j] = bf16_lo(ww);
+                        y[2 * j + 1] = bf16_hi(ww);
+                    }
+                    rht16_regs(y);
+                    bmax = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(y[j]));
+                } else {
+                    uint32_t acc = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc = absmax2(acc, w[k][j]);
+                    bmax = __uint_as_float(absmax2_fold(acc));
+                }
                 if (AMAX_ONLY) {
-                    amax_bits = max(amax_bits, __float_as_uint(bmax));
+                    if (ok[k]) amax_bits = max(amax_bits, __float_as_uint(bmax));
                     continue;
                 }
-                bmax = fmaxf(bmax, __shfl_xor_sync(0xFFFFFFFFu, bmax, 1));
-                const BlockScale bs = block_scale(bmax, t, sg);
-                const bool inf_r = isinf(bs.r);
-                float q[8];
+                if (!ok[k]) continue;
+                if (!RHT) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) q[e] = inf_r ? scaled_inf(y[e]) : scaled(y[e], bs.r);
-                if (SR) {
-                    const uint4 rb = sr_bits8(p.sr_seed, (uint64_t)(rr[k] * p.cols + cc[k]) >> 3);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) q[e] = sr_grid(q[e], sr_u16(rb, e));
-                }
-                const uint32_t packed = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-                if (ok[k]) {
-                    *reinterpret_cast<uint32_t*>(p.codes + rr[k] * (p.cols >> 1) + (cc[k] >> 1)) = packed;
-                    if ((lane & 1) == 0) {
-                        const int64_t b = cc[k] >> 4;
-                        if (p.scales) p.scales[rr[k] * kb + b] = (uint8_t)bs.code;
-                        if (p.scales_mma) p.scales_mma[mma_scale_offset(rr[k], b, p.chunks_k)] = (uint8_t)bs.code;
+                    for (int j = 0; j < 8; ++j) {
+                        y[2 * j] = bf16_lo(w[k][j]);
+                        y[2 * j + 1] = bf16_hi(w[k][j]);
                     }
                 }
+                const BlockScale bs = block_scale(bmax, t, sg);
+                uint32_t lo, hi;
+                encode16<SR>(y, bs, p.sr_seed, (uint64_t)(rr[k] * p.cols + cc[k]) >> 3, lo, hi);
+                *reinterpret_cast<uint2*>(p.codes + rr[k] * (p.cols >> 1) + (cc[k] >> 1)) = make_uint2(lo, hi);
+                const int64_t b = cc[k] >> 4;
+                if (p.scales) p.scales[rr[k] * kb + b] = (uint8_t)bs.code;
+                if (p.scales_mma) p.scales_mma[mma_scale_offset(rr[k], b, p.chunks_k)] = (uint8_t)bs.code;
             }
         }
     }
@@ -500,8 +569,8 @@ int grid_for(K kernel, int64_t work_items) {
 
 template <bool RHT, bool SR>
 cudaError_t run_rows(Params p, cudaStream_t s, int* launches) {
-    const int64_t units = p.rows * ((p.cols + 255) >> 8);
-    const int64_t warps_needed = (units + kUnroll - 1) / kUnroll;
+    const int64_t units = p.rows * ((p.cols + 511) >> 9);
+    const int64_t warps_needed = (units + 1) / 2;
     const int g = grid_for(rows_kernel<RHT, SR, false>, (warps_needed + 7) / 8);
     p.n_partials = g;
     if (RHT) {
@@ -664,8 +733,8 @@ cudaError_t launch_quantize_1d_noalloc(const QuantArgs& a, cudaStream_t s, int* 
     int g;
     const bool sr = a.rounding == 1;
     if (!a.transpose) {
-        const int64_t units = a.rows * ((a.cols + 255) >> 8);
-        const int64_t warps_needed = (units + kUnroll - 1) / kUnroll;
+        const int64_t units = a.rows * ((a.cols + 511) >> 9);
+        const int64_t warps_needed = (units + 1) / 2;
         g = sr ? grid_for(rows_kernel<false, true, false>, (warps_needed + 7) / 8)
                : grid_for(rows_kernel<false, false, false>, (warps_needed + 7) / 8);
     } else {
