@@ -36,6 +36,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -170,6 +171,67 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
+}
+
+
+// --------------------------------------------------- CTA-pair (2-SM) helpers --
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on the barrier at the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t rank) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+        ::"r"(bar), "r"(rank)
+        : "memory");
+}
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_cluster(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (mbar_try_cluster(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicExch(&g_error_word, 1u);
+            return false;
+        }
+    }
+}
+// Completion of the CTA pair's prior tcgen05 operations arrives on the barrier
+// at this offset in both CTAs.
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(bar), "h"((uint16_t)3)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
 }
 
 // Shared-memory matrix descriptor: K-major operand tile of rows x 128 bytes,
@@ -490,6 +552,312 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
 }
 
+
+// ===================================================================== 2-SM ===
+// CTA-pair variant: a cluster of two CTAs computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 64).  CTA r loads A rows
+// 128r..128r+127 and B rows 128r..128r+127 of the tile (its halves), its own
+// 128 rows of A scales and all 256 rows of B scales; its TMEM holds rows
+// 128r.. of the accumulator.  Only CTA 0 issues MMAs; their completion is
+// committed to the barriers of both CTAs.  The other CTA signals CTA 0 when
+// its scales are in TMEM (which implies its stage has landed) and when its
+// epilogue has drained the accumulator.  Per SM this moves 38 KB per 64 K
+// columns instead of 54 KB: the single-SM tile is L2-bandwidth bound.
+constexpr int P_STAGES = 5;
+constexpr int P_A_STAGE = 128 * BKB;                 // 16 KB
+constexpr int P_B_STAGE = 128 * BKB;                 // 16 KB
+constexpr int P_OFF_A = 0;
+constexpr int P_OFF_B = P_OFF_A + P_STAGES * P_A_STAGE;
+constexpr int P_OFF_SFA = P_OFF_B + P_STAGES * P_B_STAGE;
+constexpr int P_OFF_SFB = P_OFF_SFA + P_STAGES * SFA_STAGE;
+constexpr int P_OFF_BAR = P_OFF_SFB + P_STAGES * SFB_STAGE;
+constexpr int P_NUM_BARS = 2 * P_STAGES + 2 * NSF + 3;
+constexpr int P_OFF_MISC = P_OFF_BAR + P_NUM_BARS * 8;
+constexpr int P_SMEM_BYTES = P_OFF_MISC + 16 + 1024;
+// M = 256 (pair), N = 256, E2M1 x E2M1, UE4M3 scales, K-major.
+constexpr uint32_t kIdescPair = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, int half, int q, int lane, uint32_t rank,
+                                                   uint32_t tmem, float alpha, uint32_t bar_tfull, uint32_t bar_tempty,
+                                                   uint32_t& acc_phase, volatile int* abort_flag) {
+    if (!mbar_wait_cluster(bar_tfull, acc_phase, abort_flag)) return false;
+    tc_fence_after();
+    int tm, tn;
+    tile_coords(tile, p, tm, tn);
+    const int row = tm * 256 + (int)rank * 128 + q * 32 + lane;
+    const int col0 = tn * BN + half * 128;
+    const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + half * 128;
+    const int ncols = p.N - col0;
+    auto release = [&]() {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            if (rank == 0) mbar_arrive(bar_tempty);
+            else mbar_arrive_cluster(bar_tempty, 0);
+        }
+        acc_phase ^= 1;
+    };
+    if (p.out_bf16) {
+        uint32_t packed[64];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t v[16];
+            tc_ld_32x32b_x16(taddr + 16 * i, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * e]), alpha),
+                                                                __fmul_rn(__uint_as_float(v[2 * e + 1]), alpha));
+                packed[8 * i + e] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+        }
+        release();
+        if (row < p.M && ncols > 0) {
+            __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + col0;
+            if (ncols >= 128) {
+#pragma unroll
+                for (int g = 0; g < 16; ++g)
+                    *reinterpret_cast<uint4*>(crow + 8 * g) =
+                        make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+            } else {
+#pragma unroll
+                for (int g = 0; g < 64; ++g) {
+                    if (2 * g + 1 < ncols) reinterpret_cast<uint32_t*>(crow)[g] = packed[g];
+                    else if (2 * g < ncols) reinterpret_cast<uint16_t*>(crow)[2 * g] = (uint16_t)(packed[g] & 0xFFFFu);
+                }
+            }
+        }
+    } else {
+        float* crow = reinterpret_cast<float*>(p.c) + (int64_t)row * p.ldc + col0;
+#pragma unroll 1
+        for (int i = 0; i < 4; ++i) {
+            uint32_t v[32];
+            tc_ld_32x32b_x32(taddr + 32 * i, v);
+            tc_wait_ld();
+            if (row < p.M) {
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const int cc = 32 * i + 4 * g;
+                    const float4 f = make_float4(__fmul_rn(__uint_as_float(v[4 * g]), alpha),
+                                                 __fmul_rn(__uint_as_float(v[4 * g + 1]), alpha),
+                                                 __fmul_rn(__uint_as_float(v[4 * g + 2]), alpha),
+                                                 __fmul_rn(__uint_as_float(v[4 * g + 3]), alpha));
+                    if (cc + 4 <= ncols) {
+                        *reinterpret_cast<float4*>(crow + cc) = f;
+                    } else {
+                        const float ff[4] = {f.x, f.y, f.z, f.w};
+                        for (int e = 0; e < 4; ++e)
+                            if (cc + e < ncols) crow[cc + e] = ff[e];
+                    }
+                }
+            }
+        }
+        release();
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, KParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar_full = sbase + P_OFF_BAR;
+    const uint32_t bar_empty = bar_full + P_STAGES * 8;
+    const uint32_t bar_sf_full = bar_empty + P_STAGES * 8;
+    const uint32_t bar_sf_empty = bar_sf_full + NSF * 8;
+    const uint32_t bar_tfull = bar_sf_empty + NSF * 8;
+    const uint32_t bar_tempty = bar_tfull + 8;
+    const uint32_t bar_drain = bar_tempty + 8;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + P_OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P_OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+    const int k_blocks = (p.K + BK - 1) / BK;
+    const int k_steps = p.K / 64;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < P_STAGES; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        for (int b = 0; b < NSF; ++b) {
+            mbar_init(bar_sf_full + 8 * b, 8);       // 4 scale warps in each CTA
+            mbar_init(bar_sf_empty + 8 * b, 1);
+        }
+        mbar_init(bar_tfull, 1);
+        mbar_init(bar_tempty, 2 * EPI_WARPS);        // epilogue warps of both CTAs
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(TMEM_COLS));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer ----
+        if (lane == 0) {
+            int s = 0;
+            uint32_t phase = 0, issued_parity = 0, issued_any = 0;
+            bool ok = true;
+            const int rc_a_max = (p.M + 127) >> 7, rc_b_max = (p.N + 127) >> 7;
+            for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
+                int tm, tn;
+                tile_coords(tile, p, tm, tn);
+                const int m0 = tm * 256 + (int)rank * 128, n0 = tn * 256 + (int)rank * 128;
+                const int rc_a = m0 >> 7, rc_b = (tn * 256) >> 7;
+                const int has_a = rc_a < rc_a_max ? 1 : 0;
+                const int nh = (rc_b + 1 < rc_b_max) ? 2 : 1;
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait_cluster(bar_empty + 8 * s, phase ^ 1, abort_flag)) { ok = false; break; }
+                    const int nk = min(4, k_steps - kb * 4);
+                    const uint32_t full = bar_full + 8 * s;
+                    mbar_expect_tx(full, (uint32_t)(P_A_STAGE + P_B_STAGE + nk * 512 * (has_a + nh)));
+                    tma_load_2d(sbase + P_OFF_A + s * P_A_STAGE, &map_a, full, kb * BKB, m0);
+                    tma_load_2d(sbase + P_OFF_B + s * P_B_STAGE, &map_b, full, kb * BKB, n0);
+                    if (has_a)
+                        bulk_load(sbase + P_OFF_SFA + s * SFA_STAGE,
+                                  p.sfa + ((int64_t)rc_a * p.chunks_k + kb * 4) * 512, nk * 512, full);
+                    for (int h = 0; h < nh; ++h)
+                        bulk_load(sbase + P_OFF_SFB + s * SFB_STAGE + h * 2048,
+                                  p.sfb + ((int64_t)(rc_b + h) * p.chunks_k + kb * 4) * 512, nk * 512, full);
+                    issued_any |= 1u << s;
+                    issued_parity = (issued_parity & ~(1u << s)) | (phase << s);
+                    if (++s == P_STAGES) { s = 0; phase ^= 1; }
+                }
+            }
+            for (int st = 0; st < P_STAGES; ++st)
+                if (issued_any & (1u << st)) {
+                    const uint32_t par = (issued_parity >> st) & 1u;
+                    const unsigned long long t0 = globaltimer();
+                    while (!mbar_try(bar_full + 8 * st, par) && globaltimer() - t0 < kWaitLimitNs) {}
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------- MMA (CTA 0 of the pair) ----
+        if (lane == 0 && rank == 0) {
+            int s = 0, b = 0;
+            uint32_t phase = 0, bphase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
+                if (!mbar_wait_cluster(bar_tempty, acc_phase ^ 1, abort_flag)) break;
+                tc_fence_after();
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait_cluster(bar_full + 8 * s, phase, abort_flag) ||
+                        !mbar_wait_cluster(bar_sf_full + 8 * b, bphase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const int nk = min(4, k_steps - kb * 4);
+                    const uint32_t a_addr = sbase + P_OFF_A + s * P_A_STAGE;
+                    const uint32_t b_addr = sbase + P_OFF_B + s * P_B_STAGE;
+                    const uint32_t sfa_col = tmem + SF_COL + b * 48;
+                    const uint32_t sfb_col = sfa_col + 16;
+                    for (int j = 0; j < nk; ++j)
+                        tc_mma_nvf4_pair(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32),
+                                         kIdescPair, sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
+                    tc_commit_pair(bar_empty + 8 * s);
+                    tc_commit_pair(bar_sf_empty + 8 * b);
+                    if (++s == P_STAGES) { s = 0; phase ^= 1; }
+                    if (++b == NSF) { b = 0; bphase ^= 1; }
+                }
+                if (!ok) break;
+                tc_commit_pair(bar_tfull);
+                acc_phase ^= 1;
+            }
+            tc_commit_pair(bar_drain);
+        }
+        // both CTAs, also after an abort: every MMA of the pair -- and with it
+        // every commit CTA 0 multicasts to this CTA's barriers -- has completed
+        // before shared memory and TMEM can be released
+        if (lane == 0) {
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_cluster(bar_drain, 0) && globaltimer() - t0 < kWaitLimitNs) {}
+        }
+    } else if (warp < 6) {
+        // ------------------------------- scales -> TMEM, and the epilogue ----
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
+        int s = 0, b = 0;
+        uint32_t phase = 0, bphase = 0, acc_phase = 0;
+        bool ok = true;
+        int prev_tile = -1;
+        const int lead = min(4, k_blocks);
+        for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
+            for (int kb = 0; kb < k_blocks; ++kb) {
+                if (!mbar_wait_cluster(bar_full + 8 * s, phase, abort_flag) ||
+                    !mbar_wait_cluster(bar_sf_empty + 8 * b, bphase ^ 1, abort_flag)) { ok = false; break; }
+                const uint32_t sfa_s = sbase + P_OFF_SFA + s * SFA_STAGE + 16 * lane;
+                const uint32_t sfb_s = sbase + P_OFF_SFB + s * SFB_STAGE + 16 * lane;
+                uint32_t ra[16], rb0[16], rb1[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 va = lds128(sfa_s + j * 512);
+                    ra[4 * j] = va.x; ra[4 * j + 1] = va.y; ra[4 * j + 2] = va.z; ra[4 * j + 3] = va.w;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 vb = lds128(sfb_s + h * 2048 + j * 512);
+                        uint32_t* rb = j < 2 ? rb0 : rb1;
+                        const int o = 8 * (j & 1) + 4 * h;
+                        rb[o] = vb.x; rb[o + 1] = vb.y; rb[o + 2] = vb.z; rb[o + 3] = vb.w;
+                    }
+                }
+                const uint32_t col = tmem + lane_base + SF_COL + b * 48;
+                tc_st_32x32b_x16(col, ra);
+                tc_st_32x32b_x16(col + 16, rb0);
+                tc_st_32x32b_x16(col + 32, rb1);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (rank == 0) mbar_arrive(bar_sf_full + 8 * b);
+                    else mbar_arrive_cluster(bar_sf_full + 8 * b, 0);
+                }
+                if (++s == P_STAGES) { s = 0; phase ^= 1; }
+                if (++b == NSF) { b = 0; bphase ^= 1; }
+                if (kb == lead - 1 && prev_tile >= 0) {
+                    if (!epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty,
+                                            acc_phase, abort_flag)) { ok = false; break; }
+                    prev_tile = -1;
+                }
+            }
+            if (ok) prev_tile = tile;
+        }
+        if (ok && prev_tile >= 0)
+            epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag);
+    } else {
+        // ---------------------------------------- epilogue, columns 128..255 ----
+        const int q = warp & 3;
+        const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
+        uint32_t acc_phase = 0;
+        for (int tile = cluster; tile < num_tiles; tile += n_clusters)
+            if (!epilogue_half_pair(p, tile, 1, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase,
+                                    abort_flag)) break;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
+    }
+}
+
 // ----------------------------------------------------------- host side -----
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -520,26 +888,60 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t k,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count_cached() {
-    static int cached[64] = {0};
+struct DeviceInfo {
+    int sms = 0;
+    int pair_clusters = 0;   // co-resident CTA pairs of the 2-SM kernel
+};
+
+DeviceInfo device_info() {
+    static DeviceInfo cached[64];
+    static std::mutex mu;
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
-    if (!cached[dev]) {
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceInfo& d = cached[dev];
+    if (!d.sms) {
         int n = 0;
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = n > 0 ? n : 148;
         cudaFuncSetAttribute(gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaFuncSetAttribute(gemm_nvf4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+        cudaFuncSetAttribute(gemm_nvf4_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (n / 2));
+        cfg.blockDim = dim3(NUM_THREADS);
+        cfg.dynamicSmemBytes = P_SMEM_BYTES;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_nvf4_pair_kernel, &cfg) != cudaSuccess || clusters < 1) {
+            cudaGetLastError();
+            clusters = n / 2;
+        }
+        d.pair_clusters = clusters;
+        d.sms = n > 0 ? n : 148;
     }
-    return cached[dev];
+    return d;
+}
+
+int group_for(int64_t rows_per_tile, int64_t K, int tiles_m) {
+    // group as many A panels (rows_per_tile x K/2 bytes each) as fit in ~24 MB of L2
+    const int64_t panel = rows_per_tile * (K / 2);
+    int64_t gm = (24ll << 20) / (panel > 0 ? panel : 1);
+    if (gm < 1) gm = 1;
+    if (gm > tiles_m) gm = tiles_m;
+    return (int)gm;
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
-    CUtensorMap ma, mb;
-    if (!make_code_map(&ma, g.a, g.M, g.K, BM) || !make_code_map(&mb, g.b, g.N, g.K, BN))
-        return cudaErrorInvalidValue;
+    const DeviceInfo dev = device_info();
     KParams p{};
     p.sfa = g.sfa;
     p.sfb = g.sfb;
@@ -552,19 +954,43 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     p.out_bf16 = g.out_bf16;
     p.c = g.c;
     p.ldc = g.ldc;
-    p.tiles_m = (int)ceil_div(g.M, BM);
     p.tiles_n = (int)ceil_div(g.N, BN);
-    // group as many A panels (128 rows x K/2 bytes each) as fit in ~24 MB of L2
-    const int64_t panel = (int64_t)BM * (g.K / 2);
-    int64_t gm = (24ll << 20) / (panel > 0 ? panel : 1);
-    if (gm < 1) gm = 1;
-    if (gm > p.tiles_m) gm = p.tiles_m;
-    p.group_m = (int)gm;
-    const int sms = sm_count_cached();
+    // The CTA-pair kernel is kept for experiments (NVFP4_GEMM_PAIR=1): on the
+    // shapes measured so far its cross-CTA load/scale pipeline runs slower
+    // than the single-SM kernel, which is the default.
+    const char* pair = getenv("NVFP4_GEMM_PAIR");
+    if (!(pair && pair[0] == '1')) {
+        CUtensorMap ma, mb;
+        if (!make_code_map(&ma, g.a, g.M, g.K, BM) || !make_code_map(&mb, g.b, g.N, g.K, BN))
+            return cudaErrorInvalidValue;
+        p.tiles_m = (int)ceil_div(g.M, BM);
+        p.group_m = group_for(BM, g.K, p.tiles_m);
+        const int tiles = p.tiles_m * p.tiles_n;
+        const int grid = tiles < dev.sms ? tiles : dev.sms;
+        gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+        return cudaGetLastError();
+    }
+    // CTA pairs: 256 x 256 tiles, each CTA loads 128-row boxes of A and B
+    CUtensorMap ma, mb;
+    if (!make_code_map(&ma, g.a, g.M, g.K, 128) || !make_code_map(&mb, g.b, g.N, g.K, 128))
+        return cudaErrorInvalidValue;
+    p.tiles_m = (int)ceil_div(g.M, 256);
+    p.group_m = group_for(256, g.K, p.tiles_m);
     const int tiles = p.tiles_m * p.tiles_n;
-    const int grid = tiles < sms ? tiles : sms;
-    gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, p);
-    return cudaGetLastError();
+    const int clusters = tiles < dev.pair_clusters ? tiles : dev.pair_clusters;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = P_SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel, ma, mb, p);
 }
 
 unsigned int read_and_clear_error_word(cudaStream_t s, cudaError_t* err) {
