@@ -110,9 +110,13 @@ __device__ __forceinline__ uint4 sr_bits8(uint64_t seed, uint64_t g) {
     return philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), 0u, 0u), (uint32_t)seed,
                          (uint32_t)(seed >> 32));
 }
-__device__ __forceinline__ uint32_t sr_u16(const uint4& w, int e) {
+// The 16 random bits u of element e (word e/2, low half for even e), returned
+// already placed for sr_grid: ((u << 6) ^ 0x3FFFFF), i.e. ~u in bits 21..6 and
+// ones in bits 5..0.
+__device__ __forceinline__ uint32_t sr_addend(const uint4& w, int e) {
     const uint32_t word = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
-    return (e & 1) ? (word >> 16) : (word & 0xFFFFu);
+    const uint32_t placed = (e & 1) ? (word >> 10) : (word << 6);
+    return (placed & 0x3FFFC0u) ^ 0x3FFFFFu;
 }
 
 // RHT sign mask ("随机 Hadamard 变换": a random diagonal of signs): bit j set
@@ -121,25 +125,28 @@ __device__ __forceinline__ uint32_t rht_sign_mask(uint64_t rht_seed) {
     return philox4x32_10(make_uint4(0u, 0u, 1u, 0u), (uint32_t)rht_seed, (uint32_t)(rht_seed >> 32)).x & 0xFFFFu;
 }
 
-// Stochastic rounding onto the E2M1 grid of one scaled value v (|v| may be
-// +inf): between neighbours lo <= |v| < hi (gap 0.5 below 2, 1 below 4, 2
-// below 6), round up iff u < (|v| - lo) / gap * 65536 (equivalently
-// u < ceil(p * 2^16) for the integer u); |v| >= 6 gives 6.  Returns the
-// signed grid value (exactly representable in E2M1).
-__device__ __forceinline__ float sr_grid(float v, uint32_t u) {
+// Stochastic rounding onto the E2M1 grid of one scaled value v (finite):
+// between neighbours lo <= |v| < hi, p = (|v| - lo) / (hi - lo), round up iff
+// u < p * 2^16 (the same as u < ceil(p * 2^16) for the integer u); results
+// above 6 are left for the saturating E2M1 conversion.  `addend` comes from
+// sr_addend.
+//   |v| >= 1: neighbours are one E2M1 mantissa step (bit 22 of the binary32
+//     pattern) apart in every binade up to 8, and the 22 bits below it are
+//     F = p * 2^22 exactly.  bits(|v|) + (2^16 - 1 - u) * 2^6 + (2^6 - 1)
+//     carries into bit 22 iff F - 1 >= u * 2^6, i.e. iff u < p * 2^16; the
+//     carry walks into the exponent where the step doubles (1.5 -> 2, 3 -> 4).
+//   |v| < 1: the grid 0, 0.5, 1 is the grid 1, 1.5, 2 shifted by 1, so the
+//     same step runs on b = |v| + 1 rounded upwards, and 1 is taken off again.
+//     Rounding upwards to a multiple of 2^-23 moves p * 2^16 up to the next
+//     multiple of 2^-6 at most; the integer thresholds lie on that grid, so
+//     no decision changes.
+__device__ __forceinline__ float sr_grid(float v, uint32_t addend) {
     const float a = fabsf(v);
-    float q;
-    if (a >= 6.0f) {
-        q = 6.0f;
-    } else {
-        const float gap = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-        const float inv = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-        const float lo = __fmul_rn(floorf(__fmul_rn(a, inv)), gap);
-        const float frac16 = __fmul_rn(__fsub_rn(a, lo), __fmul_rn(65536.0f, inv));
-        const float uf = __fsub_rn(__uint_as_float(0x4B000000u | u), 8388608.0f);
-        q = uf < frac16 ? __fadd_rn(lo, gap) : lo;
-    }
-    return copysignf(q, v);
+    float off;
+    asm("set.lt.f32.f32 %0, %1, 0f3F800000;" : "=f"(off) : "f"(a));
+    const float b = __fadd_ru(a, off);
+    const float r = __uint_as_float((__float_as_uint(b) + addend) & 0xFFC00000u);
+    return copysignf(__fsub_rn(r, off), v);
 }
 
 // Per-block scale derived from the block amax ("精度核心:两级分层缩放";

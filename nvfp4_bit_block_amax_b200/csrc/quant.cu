@@ -181,8 +181,8 @@ __device__ __forceinline__ void encode16(const float y[16], const BlockScale& bs
         const uint4 r1 = sr_bits8(sr_seed, g + 1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            q[i] = sr_grid(q[i], sr_u16(r0, i));
-            q[i + 8] = sr_grid(q[i + 8], sr_u16(r1, i));
+            q[i] = sr_grid(q[i], sr_addend(r0, i));
+            q[i + 8] = sr_grid(q[i + 8], sr_addend(r1, i));
         }
     }
     lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
@@ -348,12 +348,13 @@ __global__ void __launch_bounds__(kThreads) cols_kernel(Params p) {
             for (int c = 0; c < 2; ++c) {
                 const int j = 2 * jp + c;
                 const BlockScale bs = block_scale(c ? bm1 : bm0, t, sg);
-                const bool inf_r = isinf(bs.r);
                 float q[16];
+                if (!isinf(bs.r)) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float yi = c ? y[i].y : y[i].x;
-                    q[i] = inf_r ? scaled_inf(yi) : scaled(yi, bs.r);
+                    for (int i = 0; i < 16; ++i) q[i] = scaled(c ? y[i].y : y[i].x, bs.r);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) q[i] = scaled_inf(c ? y[i].y : y[i].x);
                 }
                 if (SR) {
                     const uint64_t g = (uint64_t)((f0 + j) * T + t0) >> 3;
@@ -361,8 +362,8 @@ __global__ void __launch_bounds__(kThreads) cols_kernel(Params p) {
                     const uint4 r1 = sr_bits8(p.sr_seed, g + 1);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        q[i] = sr_grid(q[i], sr_u16(r0, i));
-                        q[i + 8] = sr_grid(q[i + 8], sr_u16(r1, i));
+                        q[i] = sr_grid(q[i], sr_addend(r0, i));
+                        q[i + 8] = sr_grid(q[i + 8], sr_addend(r1, i));
                     }
                 }
                 const uint32_t lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
@@ -407,12 +408,41 @@ struct Params2d {
     int n_partials;
 };
 
+// Transpose of an 8x8 matrix of nibbles held as 8 words (word i = row i,
+// nibble j = column j): afterwards word j holds column j, row i in nibble i.
+// Swaps of 4x4 blocks (16-bit halves), then 2x2 blocks (bytes), then single
+// nibbles; the three levels commute.
+__device__ __forceinline__ void transpose_nibbles8(uint32_t a[8]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t x = a[i], y = a[i + 4];
+        a[i] = __byte_perm(x, y, 0x5410);
+        a[i + 4] = __byte_perm(x, y, 0x7632);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i += (i & 1) ? 3 : 1) {   // i = 0, 1, 4, 5
+        const uint32_t x = a[i], y = a[i + 2];
+        a[i] = __byte_perm(x, y, 0x6240);
+        a[i + 2] = __byte_perm(x, y, 0x7351);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const uint32_t t = ((a[i] >> 4) ^ a[i + 1]) & 0x0F0F0F0Fu;
+        a[i + 1] ^= t;
+        a[i] ^= t << 4;
+    }
+}
+
 // CTA tile: 128 rows x 256 columns; warp w: rows 16w..16w+15, lane: 8 columns,
-// a lane pair: one 16x16 tile.  The columnwise codes (of W^T) are the same
-// element codes regrouped along rows, staged in shared memory.
+// a lane pair: one 16x16 tile.  Each lane encodes its 16 x 8 elements once
+// (row codes, one word per row); the columnwise codes (of W^T) are the same
+// nibbles transposed in registers and staged in shared memory.  The tile's
+// 128 block-scale codes are staged too, so both GEMM scale layouts are
+// written as whole 32-bit words (4 consecutive blocks of one row).
 template <bool COLS>
-__global__ void __launch_bounds__(kThreads) q2d_kernel(Params2d p) {
+__global__ void __launch_bounds__(kThreads, 2) q2d_kernel(Params2d p) {
     __shared__ __align__(16) uint8_t s_col[COLS ? 256 * 64 : 16];
+    __shared__ __align__(16) uint8_t s_sc[8][16];   // [row tile in CTA][column tile in CTA]
     float sg, t;
     {
         const float A = reduce_partials(p.partials, p.n_partials);
@@ -438,45 +468,63 @@ __global__ void __launch_bounds__(kThreads) q2d_kernel(Params2d p) {
         float b = __uint_as_float(absmax2_fold(acc));
         b = fmaxf(b, __shfl_xor_sync(0xFFFFFFFFu, b, 1));
         const BlockScale bs = block_scale(b, t, sg);
-        const bool inf_r = isinf(bs.r);
-        auto sc = [&](float x) { return inf_r ? scaled_inf(x) : scaled(x, bs.r); };
+        uint32_t rc[16];
+        if (!isinf(bs.r)) {
+            const float2 r2 = make_float2(bs.r, bs.r);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t packed =
-                e2m1x8(sc(bf16_lo(v[i].x)), sc(bf16_hi(v[i].x)), sc(bf16_lo(v[i].y)), sc(bf16_hi(v[i].y)),
-                       sc(bf16_lo(v[i].z)), sc(bf16_hi(v[i].z)), sc(bf16_lo(v[i].w)), sc(bf16_hi(v[i].w)));
-            if (ok) *reinterpret_cast<uint32_t*>(p.codes_row + (r0 + i) * (C >> 1) + (c0 >> 1)) = packed;
-        }
-        if (COLS) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float q[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const uint32_t w = (j >> 1) == 0 ? v[i].x : (j >> 1) == 1 ? v[i].y : (j >> 1) == 2 ? v[i].z : v[i].w;
-                    q[i] = sc((j & 1) ? bf16_hi(w) : bf16_lo(w));
-                }
-                const uint32_t lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-                const uint32_t hi = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
-                *reinterpret_cast<uint2*>(s_col + (lane * 8 + j) * 64 + ((warp ^ (lane & 7)) * 8)) = make_uint2(lo, hi);
+            for (int i = 0; i < 16; ++i) {
+                const float2 q0 = __fmul2_rn(make_float2(bf16_lo(v[i].x), bf16_hi(v[i].x)), r2);
+                const float2 q1 = __fmul2_rn(make_float2(bf16_lo(v[i].y), bf16_hi(v[i].y)), r2);
+                const float2 q2 = __fmul2_rn(make_float2(bf16_lo(v[i].z), bf16_hi(v[i].z)), r2);
+                const float2 q3 = __fmul2_rn(make_float2(bf16_lo(v[i].w), bf16_hi(v[i].w)), r2);
+                rc[i] = e2m1x8(q0.x, q0.y, q1.x, q1.y, q2.x, q2.y, q3.x, q3.y);
             }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                rc[i] = e2m1x8(scaled_inf(bf16_lo(v[i].x)), scaled_inf(bf16_hi(v[i].x)), scaled_inf(bf16_lo(v[i].y)),
+                               scaled_inf(bf16_hi(v[i].y)), scaled_inf(bf16_lo(v[i].z)), scaled_inf(bf16_hi(v[i].z)),
+                               scaled_inf(bf16_lo(v[i].w)), scaled_inf(bf16_hi(v[i].w)));
         }
         if (ok) {
-            const int64_t tb = c0 >> 4, trow = r0 >> 4;
-            if ((lane & 1) == 0) {
-                if (p.scales) p.scales[trow * (C >> 4) + tb] = (uint8_t)bs.code;
-                if (p.mma_row) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) p.mma_row[mma_scale_offset(r0 + i, tb, p.chunks_row)] = (uint8_t)bs.code;
-                }
+            for (int i = 0; i < 16; ++i)
+                *reinterpret_cast<uint32_t*>(p.codes_row + (r0 + i) * (C >> 1) + (c0 >> 1)) = rc[i];
+            if ((lane & 1) == 0 && p.scales) p.scales[(r0 >> 4) * (C >> 4) + (c0 >> 4)] = (uint8_t)bs.code;
+        }
+        if ((lane & 1) == 0) s_sc[warp][lane >> 1] = ok ? (uint8_t)bs.code : (uint8_t)0;
+        if (COLS) {
+            transpose_nibbles8(rc);
+            transpose_nibbles8(rc + 8);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint2*>(s_col + (lane * 8 + j) * 64 + ((warp ^ (lane & 7)) * 8)) =
+                    make_uint2(rc[j], rc[8 + j]);
+        }
+        __syncthreads();
+        // GEMM scale layouts: word = scales of blocks 4g .. 4g+3 of one row.
+        if (p.mma_row) {
+            for (int k = threadIdx.x; k < 128 * 4; k += kThreads) {
+                const int rr = k >> 2, g = k & 3;
+                const int64_t r = tr * 128 + rr, blk = tc * 16 + g * 4;
+                if (r < R && blk < (C >> 4))
+                    *reinterpret_cast<uint32_t*>(p.mma_row + mma_scale_offset(r, blk, p.chunks_row)) =
+                        *reinterpret_cast<const uint32_t*>(&s_sc[rr >> 4][g * 4]);
             }
-            if (p.mma_col) {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) p.mma_col[mma_scale_offset(c0 + j, trow, p.chunks_col)] = (uint8_t)bs.code;
+        }
+        if (p.mma_col) {
+            for (int k = threadIdx.x; k < 256 * 2; k += kThreads) {
+                const int cc = k >> 1, g = k & 1;
+                const int64_t c = tc * 256 + cc, blk = tr * 8 + g * 4;
+                if (c < C && blk < (R >> 4)) {
+                    const int cb = cc >> 4;
+                    const uint32_t word = (uint32_t)s_sc[g * 4][cb] | ((uint32_t)s_sc[g * 4 + 1][cb] << 8) |
+                                          ((uint32_t)s_sc[g * 4 + 2][cb] << 16) | ((uint32_t)s_sc[g * 4 + 3][cb] << 24);
+                    *reinterpret_cast<uint32_t*>(p.mma_col + mma_scale_offset(c, blk, p.chunks_col)) = word;
+                }
             }
         }
         if (COLS) {
-            __syncthreads();
             const int64_t cbase = tc * 256, rbyte = tr * 64;
             const int64_t row_bytes = min((int64_t)64, (R >> 1) - rbyte);
             for (int k = threadIdx.x; k < 256 * 8; k += kThreads) {
@@ -486,8 +534,8 @@ __global__ void __launch_bounds__(kThreads) q2d_kernel(Params2d p) {
                     *reinterpret_cast<uint2*>(p.codes_col + (cbase + r) * (R >> 1) + rbyte + c8 * 8) = val;
                 }
             }
-            __syncthreads();
         }
+        __syncthreads();
     }
 }
 
@@ -567,18 +615,36 @@ int grid_for(K kernel, int64_t work_items) {
     return (int)g;
 }
 
+// CTA count of the plain amax pass: up to kAmaxPerSm CTAs per SM, each with
+// kUnroll 16-byte loads per thread in flight.
+constexpr int kAmaxPerSm = 4;
+int plain_amax_grid(int64_t rows, int64_t cols) {
+    const int64_t vecs = rows * (cols >> 3);
+    const int64_t want = (vecs + (int64_t)kThreads * kUnroll - 1) / ((int64_t)kThreads * kUnroll);
+    int64_t g = std::min<int64_t>((int64_t)sm_count() * kAmaxPerSm, want);
+    g = std::max<int64_t>(g, 1);
+    return (int)std::min<int64_t>(g, kMaxPartials);
+}
+
+// Launches the plain amax pass; returns the number of partials it writes.
+int launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint32_t* partials,
+                      cudaStream_t s) {
+    const int g = plain_amax_grid(rows, cols);
+    if (ld == cols) amax_plain_kernel<true><<<g, kThreads, 0, s>>>(x, rows, cols, ld, partials);
+    else amax_plain_kernel<false><<<g, kThreads, 0, s>>>(x, rows, cols, ld, partials);
+    return g;
+}
+
 template <bool RHT, bool SR>
 cudaError_t run_rows(Params p, cudaStream_t s, int* launches) {
     const int64_t units = p.rows * ((p.cols + 511) >> 9);
     const int64_t warps_needed = (units + 1) / 2;
     const int g = grid_for(rows_kernel<RHT, SR, false>, (warps_needed + 7) / 8);
-    p.n_partials = g;
     if (RHT) {
+        p.n_partials = g;
         rows_kernel<true, false, true><<<g, kThreads, 0, s>>>(p);
     } else {
-        const bool contig = p.ld == p.cols;
-        if (contig) amax_plain_kernel<true><<<g, kThreads, 0, s>>>(p.x, p.rows, p.cols, p.ld, p.partials);
-        else amax_plain_kernel<false><<<g, kThreads, 0, s>>>(p.x, p.rows, p.cols, p.ld, p.partials);
+        p.n_partials = launch_amax_plain(p.x, p.rows, p.cols, p.ld, p.partials, s);
     }
     rows_kernel<RHT, SR, false><<<g, kThreads, 0, s>>>(p);
     *launches += 2;
@@ -589,13 +655,11 @@ template <bool RHT, bool SR>
 cudaError_t run_cols(Params p, cudaStream_t s, int* launches) {
     const int64_t tiles = ((p.rows + 127) >> 7) * ((p.cols + 255) >> 8);
     const int g = grid_for(cols_kernel<RHT, SR, false>, tiles);
-    p.n_partials = g;
     if (RHT) {
+        p.n_partials = g;
         cols_kernel<true, false, true><<<g, kThreads, 0, s>>>(p);
     } else {
-        const bool contig = p.ld == p.cols;
-        if (contig) amax_plain_kernel<true><<<g, kThreads, 0, s>>>(p.x, p.rows, p.cols, p.ld, p.partials);
-        else amax_plain_kernel<false><<<g, kThreads, 0, s>>>(p.x, p.rows, p.cols, p.ld, p.partials);
+        p.n_partials = launch_amax_plain(p.x, p.rows, p.cols, p.ld, p.partials, s);
     }
     cols_kernel<RHT, SR, false><<<g, kThreads, 0, s>>>(p);
     *launches += 2;
@@ -660,9 +724,7 @@ cudaError_t launch_quantize_2d(const Quant2dArgs& a, cudaStream_t s, int* launch
     }
     const int64_t tiles = ((a.rows + 127) >> 7) * ((a.cols + 255) >> 8);
     const int g = a.codes_col ? grid_for(q2d_kernel<true>, tiles) : grid_for(q2d_kernel<false>, tiles);
-    p.n_partials = g;
-    if (a.ld == a.cols) amax_plain_kernel<true><<<g, kThreads, 0, s>>>(a.w, a.rows, a.cols, a.ld, a.partials);
-    else amax_plain_kernel<false><<<g, kThreads, 0, s>>>(a.w, a.rows, a.cols, a.ld, a.partials);
+    p.n_partials = launch_amax_plain(a.w, a.rows, a.cols, a.ld, a.partials, s);
     if (a.codes_col) q2d_kernel<true><<<g, kThreads, 0, s>>>(p);
     else q2d_kernel<false><<<g, kThreads, 0, s>>>(p);
     *launches += 2;
@@ -722,25 +784,15 @@ cudaError_t noalloc_scratch(uint32_t** out) {
 int noalloc_capacity() { return kNoAllocPartials; }
 
 // Same launches as launch_quantize_1d, with the partial maxima in the static
-// scratch.  The CTA count of the amax pass is the one the regular path uses;
-// a configuration that would need more partials than the scratch holds is
+// scratch.  The amax pass writes one partial per CTA (plain_amax_grid); a
+// configuration that would need more partials than the scratch holds is
 // refused (*too_big = true) before anything is enqueued.
 cudaError_t launch_quantize_1d_noalloc(const QuantArgs& a, cudaStream_t s, int* launches, bool* too_big) {
     *too_big = false;
     uint32_t* scratch = nullptr;
     cudaError_t e = noalloc_scratch(&scratch);
     if (e != cudaSuccess) return e;
-    int g;
-    const bool sr = a.rounding == 1;
-    if (!a.transpose) {
-        const int64_t units = a.rows * ((a.cols + 511) >> 9);
-        const int64_t warps_needed = (units + 1) / 2;
-        g = sr ? grid_for(rows_kernel<false, true, false>, (warps_needed + 7) / 8)
-               : grid_for(rows_kernel<false, false, false>, (warps_needed + 7) / 8);
-    } else {
-        const int64_t tiles = ((a.rows + 127) >> 7) * ((a.cols + 255) >> 8);
-        g = sr ? grid_for(cols_kernel<false, true, false>, tiles) : grid_for(cols_kernel<false, false, false>, tiles);
-    }
+    const int g = plain_amax_grid(a.rows, a.cols);
     if (g > kNoAllocPartials) {
         *too_big = true;
         return cudaSuccess;
