@@ -33,13 +33,16 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Largest |bf16| of a packed pair accumulated as 16-bit unsigned magnitudes:
-// for finite values the magnitude order equals the order of (bits & 0x7FFF).
+// Largest |bf16| of a packed pair, accumulated lane-wise: max.xorsign.abs
+// keeps max(|acc|, |w|) in each half (its sign bit, the xor of the operands'
+// signs, is dropped by absmax2_fold).  Exact, subnormals included.
 __device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t w) {
-    return __vmaxu2(acc, w & 0x7FFF7FFFu);
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(acc), "r"(w));
+    return d;
 }
 __device__ __forceinline__ uint32_t absmax2_fold(uint32_t acc) {   // -> binary32 bits of the max
-    uint32_t lo = acc & 0xFFFFu, hi = acc >> 16;
+    const uint32_t lo = acc & 0x7FFFu, hi = (acc >> 16) & 0x7FFFu;
     return (lo > hi ? lo : hi) << 16;
 }
 
@@ -110,13 +113,10 @@ __device__ __forceinline__ uint4 sr_bits8(uint64_t seed, uint64_t g) {
     return philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), 0u, 0u), (uint32_t)seed,
                          (uint32_t)(seed >> 32));
 }
-// The 16 random bits u of element e (word e/2, low half for even e), returned
-// already placed for sr_grid: ((u << 6) ^ 0x3FFFFF), i.e. ~u in bits 21..6 and
-// ones in bits 5..0.
-__device__ __forceinline__ uint32_t sr_addend(const uint4& w, int e) {
+// The 16 random bits u of element e: word e/2, low half for even e.
+__device__ __forceinline__ uint32_t sr_u16(const uint4& w, int e) {
     const uint32_t word = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
-    const uint32_t placed = (e & 1) ? (word >> 10) : (word << 6);
-    return (placed & 0x3FFFC0u) ^ 0x3FFFFFu;
+    return (e & 1) ? (word >> 16) : (word & 0xFFFFu);
 }
 
 // RHT sign mask ("随机 Hadamard 变换": a random diagonal of signs): bit j set
@@ -126,27 +126,21 @@ __device__ __forceinline__ uint32_t rht_sign_mask(uint64_t rht_seed) {
 }
 
 // Stochastic rounding onto the E2M1 grid of one scaled value v (finite):
-// between neighbours lo <= |v| < hi, p = (|v| - lo) / (hi - lo), round up iff
-// u < p * 2^16 (the same as u < ceil(p * 2^16) for the integer u); results
-// above 6 are left for the saturating E2M1 conversion.  `addend` comes from
-// sr_addend.
-//   |v| >= 1: neighbours are one E2M1 mantissa step (bit 22 of the binary32
-//     pattern) apart in every binade up to 8, and the 22 bits below it are
-//     F = p * 2^22 exactly.  bits(|v|) + (2^16 - 1 - u) * 2^6 + (2^6 - 1)
-//     carries into bit 22 iff F - 1 >= u * 2^6, i.e. iff u < p * 2^16; the
-//     carry walks into the exponent where the step doubles (1.5 -> 2, 3 -> 4).
-//   |v| < 1: the grid 0, 0.5, 1 is the grid 1, 1.5, 2 shifted by 1, so the
-//     same step runs on b = |v| + 1 rounded upwards, and 1 is taken off again.
-//     Rounding upwards to a multiple of 2^-23 moves p * 2^16 up to the next
-//     multiple of 2^-6 at most; the integer thresholds lie on that grid, so
-//     no decision changes.
-__device__ __forceinline__ float sr_grid(float v, uint32_t addend) {
-    const float a = fabsf(v);
-    float off;
-    asm("set.lt.f32.f32 %0, %1, 0f3F800000;" : "=f"(off) : "f"(a));
-    const float b = __fadd_ru(a, off);
-    const float r = __uint_as_float((__float_as_uint(b) + addend) & 0xFFC00000u);
-    return copysignf(__fsub_rn(r, off), v);
+// between neighbours lo <= |v| < hi, f = floor(p * 2^16) with
+// p = (|v| - lo) / (hi - lo), round up iff f + u >= 2^16; results above 6
+// are left for the saturating E2M1 conversion.
+// E2M1 is a float with one mantissa bit and subnormals, and binary32 scaled by
+// 2^-126 lines up with it: |v| in [1, 8) becomes a normal number whose
+// mantissa bit 22 is the E2M1 mantissa bit, |v| < 1 a subnormal whose bit 22
+// is the E2M1 subnormal bit (0.5), so in both the 22 bits below bit 22 hold
+// p * 2^22, cut towards zero to an integer.  Adding u * 2^6 carries into bit
+// 22 iff floor(p * 2^22) + u * 2^6 >= 2^22, i.e. iff f + u >= 2^16 (the
+// floors nest); the carry walks into the exponent where the step doubles
+// (subnormal 0.5 -> 1, 1.5 -> 2, 3 -> 4).  Rounding towards zero keeps the
+// sign out of it, and the scaling back is exact.
+__device__ __forceinline__ float sr_grid(float v, uint32_t u) {
+    const uint32_t t = __float_as_uint(__fmul_rz(v, 0x1p-126f)) + (u << 6);
+    return __fmul_rn(__uint_as_float(t & 0xFFC00000u), 0x1p126f);
 }
 
 // Per-block scale derived from the block amax ("精度核心:两级分层缩放";
@@ -154,16 +148,49 @@ __device__ __forceinline__ float sr_grid(float v, uint32_t addend) {
 // t == 0); multiplier r = RN(1 / RN(s * s_global)).  r == 0 marks a zero
 // scale (every element encodes a signed zero); r == +inf marks a product that
 // underflowed or a reciprocal that overflowed (nonzero elements saturate).
+//
+// Per tensor, everything after the quotient depends on the 8-bit code alone,
+// so each CTA tabulates r for the 128 non-negative codes once (ScaleCtx) and
+// a block costs one quotient, one E4M3 conversion and one shared-memory load.
+// The quotient bmax / t: with y = RN(1/t), q0 = RN(bmax * y) and the exact
+// residual e = bmax - q0 * t (one FMA), RN(q0 + e * y) (one FMA) is the
+// correctly rounded quotient (Markstein's FMA division theorem) as long as
+// nothing underflows: used for t >= 2^-60, where every quotient that can
+// reach a nonzero E4M3 code (>= 2^-11) keeps e normal; IEEE division
+// otherwise.
 struct BlockScale {
     uint32_t code;
     float r;
 };
-__device__ __forceinline__ BlockScale block_scale(float bmax, float t, float sg) {
-    const float sf = (t == 0.0f) ? 0.0f : __fdiv_rn(bmax, t);
+struct ScaleCtx {
+    float t, inv_t;
+    bool fast;
+    const float* rtab;   // shared memory, 128 entries
+};
+__device__ __forceinline__ ScaleCtx make_scale_ctx(float sg, float t, float* s_rtab) {
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+        const float sdec = e4m3_decode((uint32_t)c);
+        s_rtab[c] = (sdec == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sdec, sg));
+    }
+    __syncthreads();
+    ScaleCtx c;
+    c.t = t;
+    c.fast = t >= 0x1p-60f;
+    c.inv_t = c.fast ? __frcp_rn(t) : 0.0f;
+    c.rtab = s_rtab;
+    return c;
+}
+__device__ __forceinline__ BlockScale block_scale(float bmax, const ScaleCtx& c) {
+    float sf;
+    if (c.fast) {
+        const float q0 = __fmul_rn(bmax, c.inv_t);
+        sf = __fmaf_rn(__fmaf_rn(-q0, c.t, bmax), c.inv_t, q0);
+    } else {
+        sf = (c.t == 0.0f) ? 0.0f : __fdiv_rn(bmax, c.t);
+    }
     BlockScale b;
     b.code = e4m3_encode(sf);
-    const float sdec = e4m3_decode(b.code);
-    b.r = (sdec == 0.0f) ? 0.0f : __frcp_rn(__fmul_rn(sdec, sg));
+    b.r = c.rtab[b.code & 127u];
     return b;
 }
 

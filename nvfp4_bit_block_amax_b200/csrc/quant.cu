@@ -181,8 +181,8 @@ __device__ __forceinline__ void encode16(const float y[16], const BlockScale& bs
         const uint4 r1 = sr_bits8(sr_seed, g + 1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            q[i] = sr_grid(q[i], sr_addend(r0, i));
-            q[i + 8] = sr_grid(q[i + 8], sr_addend(r1, i));
+            q[i] = sr_grid(q[i], sr_u16(r0, i));
+            q[i + 8] = sr_grid(q[i + 8], sr_u16(r1, i));
         }
     }
     lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
@@ -194,8 +194,13 @@ __device__ __forceinline__ void encode16(const float y[16], const BlockScale& bs
 // (32 blocks) per unit, consecutive units per warp, 2 units in flight.
 template <bool RHT, bool SR, bool AMAX_ONLY>
 __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
-    float sg = 0.0f, t = 0.0f;
-    if (!AMAX_ONLY) global_scales(p, sg, t);
+    __shared__ float s_rtab[128];
+    ScaleCtx ctx{};
+    if (!AMAX_ONLY) {
+        float sg, t;
+        global_scales(p, sg, t);
+        ctx = make_scale_ctx(sg, t, s_rtab);
+    }
     uint32_t sw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (RHT) {
         const uint32_t d = rht_sign_mask(p.rht_seed);
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
                     if (ok[k]) amax_bits = max(amax_bits, __float_as_uint(bmax));
                     continue;
                 }
-                if (!ok[k]) continue;
+                if (u + k >= uend) continue;   // the same for the whole warp
                 if (!RHT) {
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
@@ -271,13 +276,25 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
                         y[2 * j + 1] = bf16_hi(w[k][j]);
                     }
                 }
-                const BlockScale bs = block_scale(bmax, t, sg);
+                // Lanes past the end of the row hold zeros and encode zero
+                // scales, which is what the padded GEMM scale layout holds.
+                const BlockScale bs = block_scale(bmax, ctx);
                 uint32_t lo, hi;
                 encode16<SR>(y, bs, p.sr_seed, (uint64_t)(rr[k] * p.cols + cc[k]) >> 3, lo, hi);
-                *reinterpret_cast<uint2*>(p.codes + rr[k] * (p.cols >> 1) + (cc[k] >> 1)) = make_uint2(lo, hi);
                 const int64_t b = cc[k] >> 4;
-                if (p.scales) p.scales[rr[k] * kb + b] = (uint8_t)bs.code;
-                if (p.scales_mma) p.scales_mma[mma_scale_offset(rr[k], b, p.chunks_k)] = (uint8_t)bs.code;
+                if (ok[k]) {
+                    *reinterpret_cast<uint2*>(p.codes + rr[k] * (p.cols >> 1) + (cc[k] >> 1)) = make_uint2(lo, hi);
+                    if (p.scales) p.scales[rr[k] * kb + b] = (uint8_t)bs.code;
+                }
+                if (p.scales_mma) {
+                    // Blocks 4g .. 4g+3 of a row are 4 consecutive bytes of the
+                    // GEMM layout: lanes 4g .. 4g+3 gather them into one word.
+                    uint32_t word = bs.code;
+                    word |= __shfl_down_sync(0xFFFFFFFFu, word, 1) << 8;
+                    word |= __shfl_down_sync(0xFFFFFFFFu, word, 2) << 16;
+                    if (ok[k] && (lane & 3) == 0)
+                        *reinterpret_cast<uint32_t*>(p.scales_mma + mma_scale_offset(rr[k], b, p.chunks_k)) = word;
+                }
             }
         }
     }
@@ -293,8 +310,13 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
 template <bool RHT, bool SR, bool AMAX_ONLY>
 __global__ void __launch_bounds__(kThreads) cols_kernel(Params p) {
     __shared__ __align__(16) uint8_t s_codes[256 * 64];
-    float sg = 0.0f, t = 0.0f;
-    if (!AMAX_ONLY) global_scales(p, sg, t);
+    __shared__ float s_rtab[128];
+    ScaleCtx ctx{};
+    if (!AMAX_ONLY) {
+        float sg, t;
+        global_scales(p, sg, t);
+        ctx = make_scale_ctx(sg, t, s_rtab);
+    }
     const uint32_t dmask = RHT ? rht_sign_mask(p.rht_seed) : 0u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t T = p.rows, F = p.cols;
@@ -347,7 +369,7 @@ __global__ void __launch_bounds__(kThreads) cols_kernel(Params p) {
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 const int j = 2 * jp + c;
-                const BlockScale bs = block_scale(c ? bm1 : bm0, t, sg);
+                const BlockScale bs = block_scale(c ? bm1 : bm0, ctx);
                 float q[16];
                 if (!isinf(bs.r)) {
 #pragma unroll
@@ -362,8 +384,8 @@ __global__ void __launch_bounds__(kThreads) cols_kernel(Params p) {
                     const uint4 r1 = sr_bits8(p.sr_seed, g + 1);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        q[i] = sr_grid(q[i], sr_addend(r0, i));
-                        q[i + 8] = sr_grid(q[i + 8], sr_addend(r1, i));
+                        q[i] = sr_grid(q[i], sr_u16(r0, i));
+                        q[i + 8] = sr_grid(q[i + 8], sr_u16(r1, i));
                     }
                 }
                 const uint32_t lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
@@ -443,12 +465,13 @@ template <bool COLS>
 __global__ void __launch_bounds__(kThreads, 2) q2d_kernel(Params2d p) {
     __shared__ __align__(16) uint8_t s_col[COLS ? 256 * 64 : 16];
     __shared__ __align__(16) uint8_t s_sc[8][16];   // [row tile in CTA][column tile in CTA]
-    float sg, t;
+    __shared__ float s_rtab[128];
+    ScaleCtx ctx;
     {
         const float A = reduce_partials(p.partials, p.n_partials);
-        sg = __fdiv_rn(A, kGlobalDiv);
-        t = __fmul_rn(6.0f, sg);
+        const float sg = __fdiv_rn(A, kGlobalDiv);
         if (blockIdx.x == 0 && threadIdx.x == 0) *p.global_scale = sg;
+        ctx = make_scale_ctx(sg, __fmul_rn(6.0f, sg), s_rtab);
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t R = p.rows, C = p.cols;
@@ -467,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 2) q2d_kernel(Params2d p) {
         for (int i = 0; i < 16; ++i) acc = absmax2(absmax2(absmax2(absmax2(acc, v[i].x), v[i].y), v[i].z), v[i].w);
         float b = __uint_as_float(absmax2_fold(acc));
         b = fmaxf(b, __shfl_xor_sync(0xFFFFFFFFu, b, 1));
-        const BlockScale bs = block_scale(b, t, sg);
+        const BlockScale bs = block_scale(b, ctx);
         uint32_t rc[16];
         if (!isinf(bs.r)) {
             const float2 r2 = make_float2(bs.r, bs.r);

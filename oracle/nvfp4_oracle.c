@@ -91,10 +91,11 @@ int nvfp4o_e2m1_rne(float v) {
 }
 
 /* Stochastic rounding [P2 "随机舍入"], [P3 "Empat pengaman"]: between the two
- * neighbouring magnitudes lo <= |v| < hi, round up with probability
- * ceil(p * 2^16) / 2^16, p = (|v| - lo) / (hi - lo), using the element's 16
- * random bits u: up iff u < ceil(p * 65536).  Representable |v| never moves;
- * |v| >= 6 saturates to 6. */
+ * neighbouring magnitudes lo <= |v| < hi, p = (|v| - lo) / (hi - lo) is cut
+ * to 16 fraction bits, f = floor(p * 2^16), the element's 16 random bits u
+ * are added, and the carry decides: up iff f + u >= 2^16 (probability
+ * f / 2^16, within 2^-16 of p).  Representable |v| never moves; |v| >= 6
+ * saturates to 6. */
 int nvfp4o_e2m1_sr(float v, uint32_t u16) {
     int sign = signbit(v) ? 8 : 0;
     double a = fabs((double)v);
@@ -106,8 +107,8 @@ int nvfp4o_e2m1_sr(float v, uint32_t u16) {
     if (a == lov) return sign | lo;
     double hiv = nvfp4o_e2m1_value(lo + 1);
     double p = (a - lov) / (hiv - lov);          /* exact: the gap is a power of two */
-    double thr = ceil(p * 65536.0);
-    return sign | (((double)u16 < thr) ? lo + 1 : lo);
+    double f = floor(p * 65536.0);               /* exact: p has at most 24 significant bits */
+    return sign | ((f + (double)u16 >= 65536.0) ? lo + 1 : lo);
 }
 
 /* ------------------------------------------------------------------------ */

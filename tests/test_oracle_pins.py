@@ -169,17 +169,25 @@ def test_e2m1_sr_unbiased(v):
         p = float((a - lo) / (hi - lo))
         se = gap * np.sqrt(p * (1 - p) / n)
         assert abs(vals.mean() - float(vv)) <= 3 * se
-        # exact up-rate of the 16-bit comparison: ceil(p * 2^16) / 2^16
+        # exact up-rate of the 16-bit carry rule: floor(p * 2^16) / 2^16
         rate = np.mean(np.abs(vals) == float(hi))
-        exact = np.ceil(p * 65536) / 65536
+        exact = np.floor(p * 65536) / 65536
         assert abs(rate - exact) <= 3 * np.sqrt(exact * (1 - exact) / n)
         assert set(np.unique(np.abs(vals))) <= {float(lo), float(hi)}
 
 
-def test_sr_up_rule_is_threshold_on_16_bits():
-    # v = 0.3 -> p = 0.6, threshold ceil(0.6 * 65536) = 39322
-    thr = int(np.ceil(float(Fraction(float(F32(0.3))) / Fraction(1, 2)) * 65536))
-    assert O.e2m1_sr(0.3, thr - 1) == 1 and O.e2m1_sr(0.3, thr) == 0
+def test_sr_up_rule_is_carry_of_16_bits():
+    # v = 0.3 as binary32 (0.30000001...) lies in [0, 0.5): p = 2v, p * 65536 =
+    # 39321.60..., f = 39321; up iff f + u >= 65536, i.e. u >= 26215
+    f = int(np.floor(float(Fraction(float(F32(0.3))) / Fraction(1, 2)) * 65536))
+    assert f == 39321
+    assert O.e2m1_sr(0.3, 65536 - f - 1) == 0 and O.e2m1_sr(0.3, 65536 - f) == 1
+    assert O.e2m1_sr(-0.3, 65535) == 9 and O.e2m1_sr(-0.3, 0) == 8
+    # p just above 0: f = 0 and no u rounds up; p = 1/2^16 exactly: only u = 65535
+    tiny = F32(2.0) + F32(2.0 ** -16)          # in [2, 3): p = 2^-16
+    assert O.e2m1_sr(tiny, 65535) == 5 and O.e2m1_sr(tiny, 65534) == 4
+    below = F32(np.nextafter(F32(2.0 ** -16) * F32(0.5), F32(0)))   # p just under 2^-16 in [0, 0.5)
+    assert O.e2m1_sr(below, 65535) == 0
 
 
 # ------------------------------------------------------------ E4M3 rounding --
@@ -301,8 +309,8 @@ def _mirror_e2m1_sr(v, u):
     if CODEBOOK[lo] == a:
         return sign | lo
     p = (a - CODEBOOK[lo]) / (CODEBOOK[lo + 1] - CODEBOOK[lo])
-    thr = -((-p * 65536).numerator // (-p * 65536).denominator)  # ceil
-    return sign | (lo + 1 if u < thr else lo)
+    f = (p * 65536).numerator // (p * 65536).denominator  # floor
+    return sign | (lo + 1 if f + u >= 65536 else lo)
 
 
 def mirror_quantize_1d(x_bits, transpose=False, rht_seed=None, rounding=0, sr_seed=0):
