@@ -22,9 +22,9 @@
 //               (tcgen05.cp) issued in the same pipe costs about half an MMA.
 //   warps 2..5  one warp per TMEM lane quarter.  (a) Block scales smem ->
 //               registers -> TMEM (tcgen05.st), up to 4 K-blocks ahead of
-//               the MMAs.  (b) Once the next tile's first K-blocks have
-//               their scales, the epilogue of columns 0..127 of the
-//               finished tile.
+//               the MMAs.  (b) The epilogue of columns 0..127 of a finished
+//               tile, started the moment its accumulator is complete (the
+//               waits for scale data poll for it).
 //   warps 6..9  epilogue of columns 128..255.  Epilogue: TMEM -> registers
 //               (128 columns per thread, packed to bf16), free the
 //               accumulator for the next tile, then scale by alpha and store.
@@ -95,6 +95,18 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Non-blocking probe of a barrier phase.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -288,17 +300,24 @@ __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int ha
     const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + half * 128;
     const int ncols = p.N - col0;   // columns of this half inside C
     if (p.out_bf16) {
+        // Two rounds of 64 columns: both loads of a round are in flight
+        // before the one wait, so the accumulator is read with two TMEM
+        // round trips instead of eight.
         uint32_t packed[64];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint32_t v[16];
-            tc_ld_32x32b_x16(taddr + 16 * i, v);
+        for (int i = 0; i < 2; ++i) {
+            uint32_t v0[32], v1[32];
+            tc_ld_32x32b_x32(taddr + 64 * i, v0);
+            tc_ld_32x32b_x32(taddr + 64 * i + 32, v1);
             tc_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * e]), alpha),
-                                                                __fmul_rn(__uint_as_float(v[2 * e + 1]), alpha));
-                packed[8 * i + e] = *reinterpret_cast<const uint32_t*>(&h2);
+            for (int e = 0; e < 16; ++e) {
+                const __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v0[2 * e]), alpha),
+                                                                __fmul_rn(__uint_as_float(v0[2 * e + 1]), alpha));
+                const __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v1[2 * e]), alpha),
+                                                                __fmul_rn(__uint_as_float(v1[2 * e + 1]), alpha));
+                packed[32 * i + e] = *reinterpret_cast<const uint32_t*>(&h0);
+                packed[32 * i + 16 + e] = *reinterpret_cast<const uint32_t*>(&h1);
             }
         }
         tc_fence_before();
@@ -489,7 +508,6 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         uint32_t phase = 0, bphase = 0, acc_phase = 0;
         bool ok = true;
         int prev_tile = -1;
-        const int lead = min(4, k_blocks);   // K-blocks of the next tile prepared before the epilogue
 
         auto epilogue = [&](int tile) -> bool {
             return epilogue_half(p, tile, 0, q, lane, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag);
@@ -497,8 +515,28 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < k_blocks; ++kb) {
-                if (!mbar_wait(bar_full + 8 * s, phase, abort_flag) ||
-                    !mbar_wait(bar_sf_empty + 8 * b, bphase ^ 1, abort_flag)) { ok = false; break; }
+                // Wait for the stage and a free scale buffer; meanwhile, the
+                // moment the previous tile's accumulator is complete, drain
+                // this warp's half of it, so that the MMAs of this tile never
+                // wait on the arrival of this tile's data to get it back.
+                {
+                    const unsigned long long t0 = globaltimer();
+                    while (true) {
+                        if (prev_tile >= 0 && mbar_test(bar_tfull, acc_phase)) {
+                            if (!epilogue(prev_tile)) { ok = false; break; }
+                            prev_tile = -1;
+                        }
+                        if (mbar_test(bar_full + 8 * s, phase) && mbar_test(bar_sf_empty + 8 * b, bphase ^ 1)) break;
+                        if (*abort_flag) { ok = false; break; }
+                        if (globaltimer() - t0 > kWaitLimitNs) {
+                            *abort_flag = 1;
+                            atomicExch(&g_error_word, 1u);
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok) break;
+                }
                 const uint32_t sfa_s = sbase + OFF_SFA + s * SFA_STAGE + 16 * lane;
                 const uint32_t sfb_s = sbase + OFF_SFB + s * SFB_STAGE + 16 * lane;
                 uint32_t ra[16], rb0[16], rb1[16];
@@ -527,10 +565,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                 if (lane == 0) mbar_arrive(bar_sf_full + 8 * b);
                 if (++s == STAGES) { s = 0; phase ^= 1; }
                 if (++b == NSF) { b = 0; bphase ^= 1; }
-                if (kb == lead - 1 && prev_tile >= 0) {
-                    if (!epilogue(prev_tile)) { ok = false; break; }
-                    prev_tile = -1;
-                }
+            }
+            if (ok && prev_tile >= 0) {   // fewer K-blocks than it took the accumulator to complete
+                if (!epilogue(prev_tile)) ok = false;
+                prev_tile = -1;
             }
             if (ok) prev_tile = tile;
         }

@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
                     rht16_regs(y);
                     bmax = 0.0f;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) bmax = fmaxf(bmax, fabsf(y[j]));
+                    for (int j = 0; j < 16; j += 2) bmax = max3f(bmax, fabsf(y[j]), fabsf(y[j + 1]));
                 } else {
                     uint32_t acc = 0;
 #pragma unroll
@@ -308,8 +308,9 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
 // the RHT runs in registers.  Codes are staged in shared memory and written
 // as 8-byte row segments of Q.
 template <bool RHT, bool SR, bool AMAX_ONLY>
-__global__ void __launch_bounds__(kThreads) cols_kernel(Params p) {
-    __shared__ __align__(16) uint8_t s_codes[256 * 64];
+__global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
+    __shared__ __align__(16) uint8_t s_codes[AMAX_ONLY ? 16 : 256 * 64];
+    __shared__ __align__(16) uint8_t s_sc[AMAX_ONLY ? 1 : 256][8];   // [feature in tile][token block in tile]
     __shared__ float s_rtab[128];
     ScaleCtx ctx{};
     if (!AMAX_ONLY) {
@@ -358,50 +359,68 @@ __global__ void __launch_bounds__(kThreads) cols_kernel(Params p) {
             }
             float bm0 = 0.0f, bm1 = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                bm0 = fmaxf(bm0, fabsf(y[i].x));
-                bm1 = fmaxf(bm1, fabsf(y[i].y));
+            for (int i = 0; i < 16; i += 2) {
+                bm0 = max3f(bm0, fabsf(y[i].x), fabsf(y[i + 1].x));
+                bm1 = max3f(bm1, fabsf(y[i].y), fabsf(y[i + 1].y));
             }
             if (AMAX_ONLY) {
                 if (ok) amax_bits = max(amax_bits, __float_as_uint(fmaxf(bm0, bm1)));
                 continue;
             }
+            // Features 2jp and 2jp+1: two blocks, scaled together in f32x2.
+            const BlockScale bs0 = block_scale(bm0, ctx), bs1 = block_scale(bm1, ctx);
+            float q[2][16];
+            if (!isinf(bs0.r) && !isinf(bs1.r)) {
+                const float2 r2 = make_float2(bs0.r, bs1.r);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 v2 = __fmul2_rn(y[i], r2);
+                    q[0][i] = v2.x;
+                    q[1][i] = v2.y;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    q[0][i] = isinf(bs0.r) ? scaled_inf(y[i].x) : scaled(y[i].x, bs0.r);
+                    q[1][i] = isinf(bs1.r) ? scaled_inf(y[i].y) : scaled(y[i].y, bs1.r);
+                }
+            }
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 const int j = 2 * jp + c;
-                const BlockScale bs = block_scale(c ? bm1 : bm0, ctx);
-                float q[16];
-                if (!isinf(bs.r)) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) q[i] = scaled(c ? y[i].y : y[i].x, bs.r);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) q[i] = scaled_inf(c ? y[i].y : y[i].x);
-                }
+                const uint32_t code = c ? bs1.code : bs0.code;
                 if (SR) {
                     const uint64_t g = (uint64_t)((f0 + j) * T + t0) >> 3;
                     const uint4 r0 = sr_bits8(p.sr_seed, g);
                     const uint4 r1 = sr_bits8(p.sr_seed, g + 1);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        q[i] = sr_grid(q[i], sr_u16(r0, i));
-                        q[i + 8] = sr_grid(q[i + 8], sr_u16(r1, i));
+                        q[c][i] = sr_grid(q[c][i], sr_u16(r0, i));
+                        q[c][i + 8] = sr_grid(q[c][i + 8], sr_u16(r1, i));
                     }
                 }
-                const uint32_t lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
-                const uint32_t hi = e2m1x8(q[8], q[9], q[10], q[11], q[12], q[13], q[14], q[15]);
+                const uint32_t lo = e2m1x8(q[c][0], q[c][1], q[c][2], q[c][3], q[c][4], q[c][5], q[c][6], q[c][7]);
+                const uint32_t hi =
+                    e2m1x8(q[c][8], q[c][9], q[c][10], q[c][11], q[c][12], q[c][13], q[c][14], q[c][15]);
                 const int srow = lane * 8 + j;
                 *reinterpret_cast<uint2*>(s_codes + srow * 64 + ((warp ^ (lane & 7)) * 8)) = make_uint2(lo, hi);
-                if (ok) {
-                    const int64_t f = f0 + j, b = t0 >> 4;
-                    if (p.scales) p.scales[f * kb + b] = (uint8_t)bs.code;
-                    if (p.scales_mma) p.scales_mma[mma_scale_offset(f, b, p.chunks_k)] = (uint8_t)bs.code;
-                }
+                s_sc[srow][warp] = ok ? (uint8_t)code : (uint8_t)0;
+                if (ok && p.scales) p.scales[(f0 + j) * kb + (t0 >> 4)] = (uint8_t)code;
             }
         }
         if (AMAX_ONLY) continue;
         __syncthreads();
         const int64_t fbase = ft * 256, tbyte = tt * 64;
+        if (p.scales_mma) {
+            // GEMM scale layout: blocks 4g .. 4g+3 of a Q row are one word.
+            for (int k = threadIdx.x; k < 256 * 2; k += kThreads) {
+                const int fl = k >> 1, g = k & 1;
+                const int64_t f = fbase + fl, blk = tt * 8 + g * 4;
+                if (f < F && blk < kb)
+                    *reinterpret_cast<uint32_t*>(p.scales_mma + mma_scale_offset(f, blk, p.chunks_k)) =
+                        *reinterpret_cast<const uint32_t*>(&s_sc[fl][g * 4]);
+            }
+        }
         const int64_t row_bytes = min((int64_t)64, (T >> 1) - tbyte);
         for (int k = threadIdx.x; k < 256 * 8; k += kThreads) {
             const int r = k >> 3, c8 = k & 7;
