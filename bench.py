@@ -21,6 +21,7 @@ step on its own GPU (weak scaling, no collective on the data path).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -336,13 +337,18 @@ def native(args):
 
 
 def load_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu record, or None when
+    the record is missing or was taken on a different gemm.cu (the counters
+    then no longer describe the kernel that runs)."""
     p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
-    if os.path.exists(p):
-        try:
-            return json.load(open(p)).get("bytes_per_launch")
-        except Exception:
-            return None
-    return None
+    src = os.path.join(ROOT, "nvfp4_bit_block_amax_b200", "csrc", "gemm.cu")
+    try:
+        rec = json.load(open(p))
+        data = open(src, "rb").read()
+        sha = hashlib.sha1(b"blob %d\0" % len(data) + data).hexdigest()   # git's blob id
+        return rec.get("bytes_per_launch") if rec.get("gemm_cu_sha1") == sha else None
+    except (OSError, ValueError):
+        return None
 
 
 def e2e(torch, N, step, s, args):

@@ -201,7 +201,10 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int s
  *   c [M x ldc] FP32 or bf16 (row-major), ldc >= N.
  *   Shapes: M, N >= 1; K a multiple of 64 (K/2 bytes per code row, 16-byte
  *   aligned); ragged M and N tails are handled.  c 16-byte aligned and ldc a
- *   multiple of 8 elements. */
+ *   multiple of 8 elements.
+ *   Kernel: pairs of CTAs on two SMs computing 256 x 256 tiles (tcgen05
+ *   cta_group::2); the environment variable NVFP4_GEMM_PAIR=0 selects the
+ *   single-SM kernel (128 x 256 tiles), which meets the same tolerance. */
 nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales_mma, const float* a_gs,
                         const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_gs, int64_t M,
                         int64_t N, int64_t K, int out_dtype, void* c, int64_t ldc, void* stream);

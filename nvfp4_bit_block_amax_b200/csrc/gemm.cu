@@ -60,8 +60,11 @@ constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
 constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
-constexpr int NSF = 4;                               // scale-factor buffers in tensor memory
-constexpr int NUM_BARS = 2 * STAGES + 2 * NSF + 3;   // full, empty, sf_full, sf_empty, tmem_full/empty, drain
+// Block scales of stage s live in tensor-memory buffer s: a stage's data can
+// only land after the MMAs that read the buffer's previous contents have
+// completed (the producer waits for them), so the buffer needs no barrier of
+// its own to be freed.
+constexpr int NUM_BARS = 3 * STAGES + 3;             // full, empty, sf_full per stage; tmem_full/empty, drain
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;     // + alignment slack
 constexpr int NUM_THREADS = 320;                     // 10 warps (at most 3 per SM sub-partition)
@@ -69,8 +72,9 @@ constexpr int EPI_WARPS = 8;                         // warps 2..5: scales -> TM
                                                      // warps 6..9: epilogue columns 128..255
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;
-constexpr uint32_t SF_COL = 256;                     // NSF buffers of 48 columns (16 SFA + 32 SFB)
+constexpr uint32_t SF_COL = 256;                     // one buffer of 48 columns (16 SFA + 32 SFB) per stage
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
+static_assert(SF_COL + STAGES * 48 <= TMEM_COLS, "scale buffers must fit in tensor memory");
 
 // ------------------------------------------------------------- PTX wrappers --
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -163,13 +167,6 @@ __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[3
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
-__device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -195,12 +192,17 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive on the barrier at the same shared-memory offset in CTA `rank` of the cluster.
+// Arrive on the barrier at the same shared-memory offset in CTA `rank` of the
+// cluster.  Relaxed: what the peer waits for is tensor-memory traffic that
+// this thread has already waited out (tcgen05.wait::st / wait::ld, then
+// tcgen05.fence::before_thread_sync); a release at cluster scope would also
+// wait for every global store the warp has in flight (the epilogue's), which
+// measured above 1000 cycles per arrive.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t rank) {
     asm volatile(
         "{\n\t.reg .b32 ra;\n\t"
         "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
-        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+        "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [ra];\n\t}"
         ::"r"(bar), "r"(rank)
         : "memory");
 }
@@ -209,6 +211,17 @@ __device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) 
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -380,8 +393,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     const uint32_t bar_full = sbase + OFF_BAR;
     const uint32_t bar_empty = bar_full + STAGES * 8;
     const uint32_t bar_sf_full = bar_empty + STAGES * 8;
-    const uint32_t bar_sf_empty = bar_sf_full + NSF * 8;
-    const uint32_t bar_tfull = bar_sf_empty + NSF * 8;
+    const uint32_t bar_tfull = bar_sf_full + STAGES * 8;
     const uint32_t bar_tempty = bar_tfull + 8;
     const uint32_t bar_drain = bar_tempty + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
@@ -396,10 +408,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
-        }
-        for (int b = 0; b < NSF; ++b) {
-            mbar_init(bar_sf_full + 8 * b, 4);
-            mbar_init(bar_sf_empty + 8 * b, 1);
+            mbar_init(bar_sf_full + 8 * s, 4);
         }
         mbar_init(bar_tfull, 1);
         mbar_init(bar_tempty, EPI_WARPS);
@@ -463,28 +472,27 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         // Only MMAs go down the tensor pipe: the block scales are already in
         // tensor memory, written by the scale warps.
         if (lane == 0) {
-            int s = 0, b = 0;
-            uint32_t phase = 0, bphase = 0, acc_phase = 0;
+            int s = 0;
+            uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 if (!mbar_wait(bar_tempty, acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
                 for (int kb = 0; kb < k_blocks; ++kb) {
-                    if (!mbar_wait(bar_full + 8 * s, phase, abort_flag) ||
-                        !mbar_wait(bar_sf_full + 8 * b, bphase, abort_flag)) { ok = false; break; }
+                    // sf_full[s] is raised by the scale warps after they saw
+                    // full[s]: the stage's codes have landed too.
+                    if (!mbar_wait(bar_sf_full + 8 * s, phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const int nk = min(4, k_steps - kb * 4);
                     const uint32_t a_addr = sbase + OFF_A + s * A_STAGE;
                     const uint32_t b_addr = sbase + OFF_B + s * B_STAGE;
-                    const uint32_t sfa_col = tmem + SF_COL + b * 48;
+                    const uint32_t sfa_col = tmem + SF_COL + s * 48;
                     const uint32_t sfb_col = sfa_col + 16;
                     for (int j = 0; j < nk; ++j)
                         tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32), kIdesc,
                                     sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
                     tc_commit(bar_empty + 8 * s);
-                    tc_commit(bar_sf_empty + 8 * b);
                     if (++s == STAGES) { s = 0; phase ^= 1; }
-                    if (++b == NSF) { b = 0; bphase ^= 1; }
                 }
                 if (!ok) break;
                 tc_commit(bar_tfull);
@@ -504,8 +512,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
-        int s = 0, b = 0;
-        uint32_t phase = 0, bphase = 0, acc_phase = 0;
+        int s = 0;
+        uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
         int prev_tile = -1;
 
@@ -515,10 +523,11 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
             for (int kb = 0; kb < k_blocks; ++kb) {
-                // Wait for the stage and a free scale buffer; meanwhile, the
-                // moment the previous tile's accumulator is complete, drain
-                // this warp's half of it, so that the MMAs of this tile never
-                // wait on the arrival of this tile's data to get it back.
+                // Wait for the stage (its scale buffer is free by then);
+                // meanwhile, the moment the previous tile's accumulator is
+                // complete, drain this warp's half of it, so that the MMAs of
+                // this tile never wait on the arrival of this tile's data to
+                // get it back.
                 {
                     const unsigned long long t0 = globaltimer();
                     while (true) {
@@ -526,7 +535,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                             if (!epilogue(prev_tile)) { ok = false; break; }
                             prev_tile = -1;
                         }
-                        if (mbar_test(bar_full + 8 * s, phase) && mbar_test(bar_sf_empty + 8 * b, bphase ^ 1)) break;
+                        if (mbar_test(bar_full + 8 * s, phase)) break;
                         if (*abort_flag) { ok = false; break; }
                         if (globaltimer() - t0 > kWaitLimitNs) {
                             *abort_flag = 1;
@@ -555,16 +564,15 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                         rb[o] = vb.x; rb[o + 1] = vb.y; rb[o + 2] = vb.z; rb[o + 3] = vb.w;
                     }
                 }
-                const uint32_t col = tmem + lane_base + SF_COL + b * 48;
+                const uint32_t col = tmem + lane_base + SF_COL + s * 48;
                 tc_st_32x32b_x16(col, ra);
                 tc_st_32x32b_x16(col + 16, rb0);
                 tc_st_32x32b_x16(col + 32, rb1);
                 tc_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar_sf_full + 8 * b);
+                if (lane == 0) mbar_arrive(bar_sf_full + 8 * s);
                 if (++s == STAGES) { s = 0; phase ^= 1; }
-                if (++b == NSF) { b = 0; bphase ^= 1; }
             }
             if (ok && prev_tile >= 0) {   // fewer K-blocks than it took the accumulator to complete
                 if (!epilogue(prev_tile)) ok = false;
@@ -602,6 +610,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 // epilogue has drained the accumulator.  Per SM this moves 38 KB per 64 K
 // columns instead of 54 KB: the single-SM tile is L2-bandwidth bound.
 constexpr int P_STAGES = 5;
+static_assert(SF_COL + P_STAGES * 48 <= TMEM_COLS, "scale buffers must fit in tensor memory");
 constexpr int P_A_STAGE = 128 * BKB;                 // 16 KB
 constexpr int P_B_STAGE = 128 * BKB;                 // 16 KB
 constexpr int P_OFF_A = 0;
@@ -609,7 +618,7 @@ constexpr int P_OFF_B = P_OFF_A + P_STAGES * P_A_STAGE;
 constexpr int P_OFF_SFA = P_OFF_B + P_STAGES * P_B_STAGE;
 constexpr int P_OFF_SFB = P_OFF_SFA + P_STAGES * SFA_STAGE;
 constexpr int P_OFF_BAR = P_OFF_SFB + P_STAGES * SFB_STAGE;
-constexpr int P_NUM_BARS = 2 * P_STAGES + 2 * NSF + 3;
+constexpr int P_NUM_BARS = 3 * P_STAGES + 3;   // full, empty, sf_full per stage; tmem_full/empty, drain
 constexpr int P_OFF_MISC = P_OFF_BAR + P_NUM_BARS * 8;
 constexpr int P_SMEM_BYTES = P_OFF_MISC + 16 + 1024;
 // M = 256 (pair), N = 256, E2M1 x E2M1, UE4M3 scales, K-major.
@@ -638,15 +647,19 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
     if (p.out_bf16) {
         uint32_t packed[64];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint32_t v[16];
-            tc_ld_32x32b_x16(taddr + 16 * i, v);
+        for (int i = 0; i < 2; ++i) {   // two TMEM round trips of 64 columns
+            uint32_t v0[32], v1[32];
+            tc_ld_32x32b_x32(taddr + 64 * i, v0);
+            tc_ld_32x32b_x32(taddr + 64 * i + 32, v1);
             tc_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[2 * e]), alpha),
-                                                                __fmul_rn(__uint_as_float(v[2 * e + 1]), alpha));
-                packed[8 * i + e] = *reinterpret_cast<const uint32_t*>(&h2);
+            for (int e = 0; e < 16; ++e) {
+                const __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v0[2 * e]), alpha),
+                                                                __fmul_rn(__uint_as_float(v0[2 * e + 1]), alpha));
+                const __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v1[2 * e]), alpha),
+                                                                __fmul_rn(__uint_as_float(v1[2 * e + 1]), alpha));
+                packed[32 * i + e] = *reinterpret_cast<const uint32_t*>(&h0);
+                packed[32 * i + 16 + e] = *reinterpret_cast<const uint32_t*>(&h1);
             }
         }
         release();
@@ -703,8 +716,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     const uint32_t bar_full = sbase + P_OFF_BAR;
     const uint32_t bar_empty = bar_full + P_STAGES * 8;
     const uint32_t bar_sf_full = bar_empty + P_STAGES * 8;
-    const uint32_t bar_sf_empty = bar_sf_full + NSF * 8;
-    const uint32_t bar_tfull = bar_sf_empty + NSF * 8;
+    const uint32_t bar_tfull = bar_sf_full + P_STAGES * 8;
     const uint32_t bar_tempty = bar_tfull + 8;
     const uint32_t bar_drain = bar_tempty + 8;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + P_OFF_MISC);
@@ -721,10 +733,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
         for (int s = 0; s < P_STAGES; ++s) {
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
-        }
-        for (int b = 0; b < NSF; ++b) {
-            mbar_init(bar_sf_full + 8 * b, 8);       // 4 scale warps in each CTA
-            mbar_init(bar_sf_empty + 8 * b, 1);
+            mbar_init(bar_sf_full + 8 * s, 8);       // 4 scale warps in each CTA
         }
         mbar_init(bar_tfull, 1);
         mbar_init(bar_tempty, 2 * EPI_WARPS);        // epilogue warps of both CTAs
@@ -786,28 +795,27 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     } else if (warp == 1) {
         // ------------------------------------------- MMA (CTA 0 of the pair) ----
         if (lane == 0 && rank == 0) {
-            int s = 0, b = 0;
-            uint32_t phase = 0, bphase = 0, acc_phase = 0;
+            int s = 0;
+            uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
                 if (!mbar_wait_cluster(bar_tempty, acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
                 for (int kb = 0; kb < k_blocks; ++kb) {
-                    if (!mbar_wait_cluster(bar_full + 8 * s, phase, abort_flag) ||
-                        !mbar_wait_cluster(bar_sf_full + 8 * b, bphase, abort_flag)) { ok = false; break; }
+                    // raised by the scale warps of both CTAs once their own
+                    // stage s had landed
+                    if (!mbar_wait_cluster(bar_sf_full + 8 * s, phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const int nk = min(4, k_steps - kb * 4);
                     const uint32_t a_addr = sbase + P_OFF_A + s * P_A_STAGE;
                     const uint32_t b_addr = sbase + P_OFF_B + s * P_B_STAGE;
-                    const uint32_t sfa_col = tmem + SF_COL + b * 48;
+                    const uint32_t sfa_col = tmem + SF_COL + s * 48;
                     const uint32_t sfb_col = sfa_col + 16;
                     for (int j = 0; j < nk; ++j)
                         tc_mma_nvf4_pair(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32),
                                          kIdescPair, sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
                     tc_commit_pair(bar_empty + 8 * s);
-                    tc_commit_pair(bar_sf_empty + 8 * b);
                     if (++s == P_STAGES) { s = 0; phase ^= 1; }
-                    if (++b == NSF) { b = 0; bphase ^= 1; }
                 }
                 if (!ok) break;
                 tc_commit_pair(bar_tfull);
@@ -827,15 +835,33 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
-        int s = 0, b = 0;
-        uint32_t phase = 0, bphase = 0, acc_phase = 0;
+        int s = 0;
+        uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
         int prev_tile = -1;
-        const int lead = min(4, k_blocks);
         for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
             for (int kb = 0; kb < k_blocks; ++kb) {
-                if (!mbar_wait_cluster(bar_full + 8 * s, phase, abort_flag) ||
-                    !mbar_wait_cluster(bar_sf_empty + 8 * b, bphase ^ 1, abort_flag)) { ok = false; break; }
+                // As in the single-SM kernel: wait for the stage, draining the
+                // previous tile's accumulator half the moment it is complete.
+                {
+                    const unsigned long long t0 = globaltimer();
+                    while (true) {
+                        if (prev_tile >= 0 && mbar_test_cluster(bar_tfull, acc_phase)) {
+                            if (!epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty,
+                                                    acc_phase, abort_flag)) { ok = false; break; }
+                            prev_tile = -1;
+                        }
+                        if (mbar_test_cluster(bar_full + 8 * s, phase)) break;
+                        if (*abort_flag) { ok = false; break; }
+                        if (globaltimer() - t0 > kWaitLimitNs) {
+                            *abort_flag = 1;
+                            atomicExch(&g_error_word, 1u);
+                            ok = false;
+                            break;
+                        }
+                    }
+                    if (!ok) break;
+                }
                 const uint32_t sfa_s = sbase + P_OFF_SFA + s * SFA_STAGE + 16 * lane;
                 const uint32_t sfb_s = sbase + P_OFF_SFB + s * SFB_STAGE + 16 * lane;
                 uint32_t ra[16], rb0[16], rb1[16];
@@ -854,7 +880,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                         rb[o] = vb.x; rb[o + 1] = vb.y; rb[o + 2] = vb.z; rb[o + 3] = vb.w;
                     }
                 }
-                const uint32_t col = tmem + lane_base + SF_COL + b * 48;
+                const uint32_t col = tmem + lane_base + SF_COL + s * 48;
                 tc_st_32x32b_x16(col, ra);
                 tc_st_32x32b_x16(col + 16, rb0);
                 tc_st_32x32b_x16(col + 32, rb1);
@@ -862,16 +888,15 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    if (rank == 0) mbar_arrive(bar_sf_full + 8 * b);
-                    else mbar_arrive_cluster(bar_sf_full + 8 * b, 0);
+                    if (rank == 0) mbar_arrive(bar_sf_full + 8 * s);
+                    else mbar_arrive_cluster(bar_sf_full + 8 * s, 0);
                 }
                 if (++s == P_STAGES) { s = 0; phase ^= 1; }
-                if (++b == NSF) { b = 0; bphase ^= 1; }
-                if (kb == lead - 1 && prev_tile >= 0) {
-                    if (!epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty,
-                                            acc_phase, abort_flag)) { ok = false; break; }
-                    prev_tile = -1;
-                }
+            }
+            if (ok && prev_tile >= 0) {
+                if (!epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase,
+                                        abort_flag)) ok = false;
+                prev_tile = -1;
             }
             if (ok) prev_tile = tile;
         }
@@ -993,11 +1018,11 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     p.c = g.c;
     p.ldc = g.ldc;
     p.tiles_n = (int)ceil_div(g.N, BN);
-    // The CTA-pair kernel is kept for experiments (NVFP4_GEMM_PAIR=1): on the
-    // shapes measured so far its cross-CTA load/scale pipeline runs slower
-    // than the single-SM kernel, which is the default.
+    // The CTA-pair kernel is the default: per SM it moves 38 KB instead of
+    // 54 KB from L2 per 256-wide K block.  NVFP4_GEMM_PAIR=0 selects the
+    // single-SM kernel, as does a device on which no pair can be co-resident.
     const char* pair = getenv("NVFP4_GEMM_PAIR");
-    if (!(pair && pair[0] == '1')) {
+    if ((pair && pair[0] == '0') || dev.pair_clusters < 1) {
         CUtensorMap ma, mb;
         if (!make_code_map(&ma, g.a, g.M, g.K, BM) || !make_code_map(&mb, g.b, g.N, g.K, BN))
             return cudaErrorInvalidValue;

@@ -15,6 +15,14 @@ TOL = 2e-3
 WORST = {}
 
 
+@pytest.fixture(params=["pair", "single_sm"], autouse=True)
+def gemm_kernel(request, monkeypatch):
+    """Every GEMM test runs on both kernels: the CTA-pair kernel (default)
+    and the single-SM kernel (NVFP4_GEMM_PAIR=0)."""
+    monkeypatch.setenv("NVFP4_GEMM_PAIR", "1" if request.param == "pair" else "0")
+    return request.param
+
+
 def bf16_half_ulp(x):
     """Half a bf16 unit in the last place at |x| (the store rounding of a bf16 output)."""
     x = np.abs(np.asarray(x, dtype=np.float64))
