@@ -51,7 +51,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default=None,
-                    choices=["gemm", "quantize_1d", "quantize_1d_sr", "quantize_2d", "rht_t_sr", "rht_t_rne",
+                    choices=["gemm", "gemm_amax", "quantize_1d", "quantize_1d_sr", "quantize_2d", "rht_t_sr",
+                             "rht_t_rne", "quantize_1d_from_amax", "quantize_2d_from_amax",
                              "dequantize"],
                     help="time one kernel family alone on --shape (profiling mode)")
     ap.add_argument("--shape", default=None, help="M,N,K for gemm; rows,cols otherwise")
@@ -479,7 +480,7 @@ def micro(args):
     g = torch.Generator(device=dev)
     g.manual_seed(1234)
     s = torch.cuda.Stream(device=dev)
-    if args.op == "gemm":
+    if args.op in ("gemm", "gemm_amax"):
         M, Nn, K = dims
         a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
         b = torch.randint(0, 256, (Nn, K // 2), dtype=torch.uint8, device=dev, generator=g)
@@ -487,7 +488,12 @@ def micro(args):
         sb = torch.randint(0x30, 0x40, (N.nvfp4_mma_scale_bytes(Nn, K),), dtype=torch.uint8, device=dev, generator=g)
         gs = torch.ones(2, dtype=torch.float32, device=dev)
         c = torch.empty(M, Nn, dtype=torch.bfloat16, device=dev)
-        fn = lambda: N.nvfp4_gemm(a, sa, gs[0:1], b, sb, gs[1:2], M, Nn, K, N.NVFP4_OUT_BF16, c, Nn, s)
+        if args.op == "gemm_amax":
+            camax = torch.empty(1, dtype=torch.float32, device=dev)
+            fn = lambda: N.nvfp4_gemm_amax(a, sa, gs[0:1], b, sb, gs[1:2], M, Nn, K, N.NVFP4_OUT_BF16, c, Nn,
+                                           camax, s)
+        else:
+            fn = lambda: N.nvfp4_gemm(a, sa, gs[0:1], b, sb, gs[1:2], M, Nn, K, N.NVFP4_OUT_BF16, c, Nn, s)
         work, unit = 2.0 * M * Nn * K, "TFLOP/s"
     else:
         R, C = dims
@@ -503,6 +509,16 @@ def micro(args):
             rnd = N.NVFP4_SR if args.op.endswith("sr") else N.NVFP4_RNE
             fn = lambda: N.nvfp4_quantize_1d(x, R, C, C, 0, rnd, 7, codes, None, smma, gs, ws, ws.numel(), s)
             work = R * C * (2 + 0.5 + 1 / 16)
+        elif args.op == "quantize_1d_from_amax":
+            amax = x.float().abs().max().reshape(1).contiguous()
+            fn = lambda: N.nvfp4_quantize_1d_from_amax(x, R, C, C, 0, N.NVFP4_RNE, 7, amax, codes, None, smma, gs, s)
+            work = R * C * (2 + 0.5 + 1 / 16)
+        elif args.op == "quantize_2d_from_amax":
+            amax = x.float().abs().max().reshape(1).contiguous()
+            cc = torch.empty(C, R // 2, dtype=torch.uint8, device=dev)
+            sm2 = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)
+            fn = lambda: N.nvfp4_quantize_2d_from_amax(x, R, C, C, amax, codes, cc, None, smma, sm2, gs, s)
+            work = R * C * (2 + 0.5 + 0.5 + 2 / 16)
         elif args.op == "quantize_2d":
             cc = torch.empty(C, R // 2, dtype=torch.uint8, device=dev)
             sm2 = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)

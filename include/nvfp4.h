@@ -97,7 +97,10 @@ size_t nvfp4_mma_scale_bytes(int64_t rows, int64_t k);
  *   rounding   NVFP4_RNE or NVFP4_SR.  SR draws 16 bits per element from
  *              Philox4x32-10 keyed by sr_seed at counter (i/8, 0) where i is
  *              the element's index in Q (row-major); word (i%8)/2, low half
- *              for even i; round up iff bits < ceil(p * 65536).
+ *              for even i.  Between the neighbouring codes lo <= |v| < hi,
+ *              p = (|v| - lo) / (hi - lo): round up iff floor(p * 65536) + bits
+ *              >= 65536 (the carry of the random bits added below the kept
+ *              precision; up-rate within 2^-16 of p).
  *   Outputs for Q of shape [Qr x Qc] (Qc % 16 == 0):
  *     codes        [Qr x Qc/2] packed E2M1 (required),
  *     scales       [Qr x Qc/16] E4M3, plain layout (nullable),
@@ -129,9 +132,10 @@ nvfp4_status nvfp4_quantize_1d(const void* x, int64_t rows, int64_t cols, int64_
  *   - The first call on a device looks up that array's device address (once
  *     per device, with that device current); make this first call before any
  *     stream capture.
- *   - A call whose amax pass would need more than 1024 partials (more CTAs
- *     than a 148-SM B200 launches for this kernel) is refused with
- *     NVFP4_ERR_WORKSPACE before anything is enqueued.
+ *   - The amax pass launches at most 4 CTAs per SM, one partial each; on a
+ *     device with more than 256 SMs a call that would need more than 1024
+ *     partials is refused with NVFP4_ERR_WORKSPACE before anything is
+ *     enqueued.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents; each call's amax pass overwrites every entry its encode pass
  *     reads, so nothing needs clearing between calls.  Calls that overlap on
@@ -179,6 +183,26 @@ nvfp4_status nvfp4_quantize_2d(const void* w, int64_t rows, int64_t cols, int64_
                                uint8_t* scales_mma_col, float* global_scale, void* workspace,
                                size_t ws_bytes, void* stream);
 
+/* Quantization with the tensor amax already known ["NVFP4 Is a Scaling
+ * System, Not Just a 4-Bit Number", "Where speed and accuracy claims can
+ * fail" -- quantization and scale handling consume work]: the amax pass,
+ * i.e. the first full read of the input, is skipped.  The amax typically comes
+ * from the kernel that produced the input (nvfp4_gemm_amax).
+ *   amax  device pointer to max |x| over the tensor as it will be quantized
+ *         (finite, >= 0).  The result is bit-identical to nvfp4_quantize_1d /
+ *         nvfp4_quantize_2d when amax is exact; a larger value gives a valid
+ *         but coarser quantization, a smaller one saturates codes at +-6.
+ *   No workspace.  Other arguments and outputs as nvfp4_quantize_1d /
+ *   nvfp4_quantize_2d (there is no RHT variant: the amax of the rotated
+ *   tensor is not known to a producer). */
+nvfp4_status nvfp4_quantize_1d_from_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                                         int rounding, uint64_t sr_seed, const float* amax, uint8_t* codes,
+                                         uint8_t* scales, uint8_t* scales_mma, float* global_scale, void* stream);
+nvfp4_status nvfp4_quantize_2d_from_amax(const void* w, int64_t rows, int64_t cols, int64_t ld, const float* amax,
+                                         uint8_t* codes_row, uint8_t* codes_col, uint8_t* scales,
+                                         uint8_t* scales_mma_row, uint8_t* scales_mma_col, float* global_scale,
+                                         void* stream);
+
 /* Reconstruction x = value(code) * s_block * s_global ["The smallest example:
  * the same payload, two real values"]: out = RN(RN(value * s_block) *
  * s_global) in binary32 (the inner product is exact); NVFP4_OUT_BF16 rounds
@@ -209,6 +233,18 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales_mma, con
                         const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_gs, int64_t M,
                         int64_t N, int64_t K, int out_dtype, void* c, int64_t ldc, void* stream);
 
+/* nvfp4_gemm that also produces the tensor amax of its output, so that the
+ * next layer can quantize C in one read (nvfp4_quantize_1d_from_amax) ["NVFP4
+ * Is a Scaling System, Not Just a 4-Bit Number", "Where speed and accuracy
+ * claims can fail"]: c_amax (device float, 4-byte aligned) receives max |C|
+ * over the M x N stored values (after the bf16 rounding for a bf16 C).  The
+ * library zeroes it first, then every epilogue warp folds its maximum in with
+ * one atomic. */
+nvfp4_status nvfp4_gemm_amax(const uint8_t* a_codes, const uint8_t* a_scales_mma, const float* a_gs,
+                             const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_gs, int64_t M,
+                             int64_t N, int64_t K, int out_dtype, void* c, int64_t ldc, float* c_amax,
+                             void* stream);
+
 /* Re-layout plain scales into the MMA layout (for callers that kept only the
  * plain layout).  scale_mode 1D: scales [rows x k/16]; 2D: [rows/16 x k/16],
  * expanded per row.  scales_mma: nvfp4_mma_scale_bytes(rows, k) bytes. */
@@ -224,6 +260,16 @@ long long nvfp4_kernel_launches(void);
  * library traps or spins without bound.  Returns NVFP4_ERR_CUDA if the stream
  * itself reports an error. */
 nvfp4_status nvfp4_get_error(void* stream);
+
+/* Self-test of the failure path (no counterpart on the pages): enqueues one
+ * small kernel in which a thread waits, bounded by `limit_ns` nanoseconds, on
+ * a barrier that nothing arrives on -- the same bounded wait every pipeline
+ * barrier of the GEMM uses.  When the limit runs out the kernel raises the
+ * device error word and returns normally, so the next nvfp4_get_error on the
+ * stream reports NVFP4_ERR_TIMEOUT and clears it; the context stays usable.
+ * No fault, trap or unbounded spin is involved.
+ *   limit_ns in [1000, 2e9], else NVFP4_ERR_INVALID_ARG. */
+nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 #ifdef __cplusplus
 }

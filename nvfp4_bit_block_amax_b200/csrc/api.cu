@@ -71,7 +71,7 @@ long long nvfp4_kernel_launches(void) { return g_launches.load(); }
 static nvfp4_status quantize_1d_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose, int rht,
                                      uint64_t rht_seed, int rounding, uint64_t sr_seed, uint8_t* codes,
                                      uint8_t* scales, uint8_t* scales_mma, float* global_scale, void* workspace,
-                                     size_t ws_bytes, void* stream) {
+                                     size_t ws_bytes, void* stream, const float* given_amax = nullptr) {
     nvfp4_status st = check_quant_common(x, rows, cols, ld, transpose, rounding, codes, scales, scales_mma,
                                          global_scale, workspace, ws_bytes);
     if (st != NVFP4_OK) return st;
@@ -90,6 +90,7 @@ static nvfp4_status quantize_1d_impl(const void* x, int64_t rows, int64_t cols, 
     a.scales_mma = scales_mma;
     a.global_scale = global_scale;
     a.partials = static_cast<uint32_t*>(workspace);
+    a.given_amax = given_amax;
     int n = 0;
     cudaError_t e = launch_quantize_1d(a, static_cast<cudaStream_t>(stream), &n);
     g_launches += n;
@@ -101,6 +102,16 @@ nvfp4_status nvfp4_quantize_1d(const void* x, int64_t rows, int64_t cols, int64_
                                float* global_scale, void* workspace, size_t ws_bytes, void* stream) {
     return quantize_1d_impl(x, rows, cols, ld, transpose, 0, 0, rounding, sr_seed, codes, scales, scales_mma,
                             global_scale, workspace, ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_quantize_1d_from_amax(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                                         int rounding, uint64_t sr_seed, const float* amax, uint8_t* codes,
+                                         uint8_t* scales, uint8_t* scales_mma, float* global_scale, void* stream) {
+    if (!amax) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned4(amax)) return NVFP4_ERR_MISALIGNED;
+    // no amax pass, so no workspace: the check gets a placeholder it only compares
+    return quantize_1d_impl(x, rows, cols, ld, transpose, 0, 0, rounding, sr_seed, codes, scales, scales_mma,
+                            global_scale, reinterpret_cast<void*>(uintptr_t(256)), kWorkspaceBytes, stream, amax);
 }
 
 nvfp4_status nvfp4_quantize_1d_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
@@ -141,10 +152,10 @@ nvfp4_status nvfp4_rht_quantize_sr(const void* x, int64_t rows, int64_t cols, in
                             scales_mma, global_scale, workspace, ws_bytes, stream);
 }
 
-nvfp4_status nvfp4_quantize_2d(const void* w, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes_row,
-                               uint8_t* codes_col, uint8_t* scales, uint8_t* scales_mma_row,
-                               uint8_t* scales_mma_col, float* global_scale, void* workspace, size_t ws_bytes,
-                               void* stream) {
+static nvfp4_status quantize_2d_impl(const void* w, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes_row,
+                                     uint8_t* codes_col, uint8_t* scales, uint8_t* scales_mma_row,
+                                     uint8_t* scales_mma_col, float* global_scale, void* workspace,
+                                     size_t ws_bytes, void* stream, const float* given_amax) {
     if (!w || !codes_row || !global_scale || (!scales && !scales_mma_row && !scales_mma_col))
         return NVFP4_ERR_INVALID_ARG;
     if (rows < 1 || cols < 1 || ld < cols || rows >= kMaxDim || cols >= kMaxDim) return NVFP4_ERR_INVALID_ARG;
@@ -166,10 +177,29 @@ nvfp4_status nvfp4_quantize_2d(const void* w, int64_t rows, int64_t cols, int64_
     a.scales_mma_col = scales_mma_col;
     a.global_scale = global_scale;
     a.partials = static_cast<uint32_t*>(workspace);
+    a.given_amax = given_amax;
     int n = 0;
     cudaError_t e = launch_quantize_2d(a, static_cast<cudaStream_t>(stream), &n);
     g_launches += n;
     return from_cuda(e);
+}
+
+nvfp4_status nvfp4_quantize_2d(const void* w, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes_row,
+                               uint8_t* codes_col, uint8_t* scales, uint8_t* scales_mma_row,
+                               uint8_t* scales_mma_col, float* global_scale, void* workspace, size_t ws_bytes,
+                               void* stream) {
+    return quantize_2d_impl(w, rows, cols, ld, codes_row, codes_col, scales, scales_mma_row, scales_mma_col,
+                            global_scale, workspace, ws_bytes, stream, nullptr);
+}
+
+nvfp4_status nvfp4_quantize_2d_from_amax(const void* w, int64_t rows, int64_t cols, int64_t ld, const float* amax,
+                                         uint8_t* codes_row, uint8_t* codes_col, uint8_t* scales,
+                                         uint8_t* scales_mma_row, uint8_t* scales_mma_col, float* global_scale,
+                                         void* stream) {
+    if (!amax) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned4(amax)) return NVFP4_ERR_MISALIGNED;
+    return quantize_2d_impl(w, rows, cols, ld, codes_row, codes_col, scales, scales_mma_row, scales_mma_col,
+                            global_scale, reinterpret_cast<void*>(uintptr_t(256)), kWorkspaceBytes, stream, amax);
 }
 
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int scale_mode,
@@ -187,9 +217,10 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int s
     return from_cuda(e);
 }
 
-nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales_mma, const float* a_gs,
-                        const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_gs, int64_t M,
-                        int64_t N, int64_t K, int out_dtype, void* c, int64_t ldc, void* stream) {
+static nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales_mma, const float* a_gs,
+                              const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_gs, int64_t M,
+                              int64_t N, int64_t K, int out_dtype, void* c, int64_t ldc, float* c_amax,
+                              void* stream) {
     if (!a_codes || !a_scales_mma || !a_gs || !b_codes || !b_scales_mma || !b_gs || !c)
         return NVFP4_ERR_INVALID_ARG;
     if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
@@ -212,9 +243,31 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales_mma, con
     g.out_bf16 = out_dtype == NVFP4_OUT_BF16;
     g.c = c;
     g.ldc = ldc;
+    g.c_amax = c_amax;
+    if (c_amax) {
+        cudaError_t z = cudaMemsetAsync(c_amax, 0, sizeof(float), static_cast<cudaStream_t>(stream));
+        if (z != cudaSuccess) return NVFP4_ERR_CUDA;
+    }
     cudaError_t e = launch_gemm(g, static_cast<cudaStream_t>(stream));
     g_launches += 1;
     return from_cuda(e);
+}
+
+nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales_mma, const float* a_gs,
+                        const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_gs, int64_t M,
+                        int64_t N, int64_t K, int out_dtype, void* c, int64_t ldc, void* stream) {
+    return gemm_impl(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K, out_dtype, c, ldc, nullptr,
+                     stream);
+}
+
+nvfp4_status nvfp4_gemm_amax(const uint8_t* a_codes, const uint8_t* a_scales_mma, const float* a_gs,
+                             const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_gs, int64_t M,
+                             int64_t N, int64_t K, int out_dtype, void* c, int64_t ldc, float* c_amax,
+                             void* stream) {
+    if (!c_amax) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned4(c_amax)) return NVFP4_ERR_MISALIGNED;
+    return gemm_impl(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K, out_dtype, c, ldc, c_amax,
+                     stream);
 }
 
 nvfp4_status nvfp4_scales_to_mma(const uint8_t* scales, int scale_mode, int64_t rows, int64_t k,
@@ -226,6 +279,14 @@ nvfp4_status nvfp4_scales_to_mma(const uint8_t* scales, int scale_mode, int64_t 
     cudaError_t e = launch_scales_to_mma(scales, scale_mode, rows, k, scales_mma, static_cast<cudaStream_t>(stream));
     g_launches += 1;
     return from_cuda(e);
+}
+
+nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, void* stream) {
+    if (limit_ns < 1000 || limit_ns > 2000000000ull) return NVFP4_ERR_INVALID_ARG;
+    g_launches.fetch_add(1);
+    return launch_wait_selftest((unsigned long long)limit_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? NVFP4_OK
+               : NVFP4_ERR_CUDA;
 }
 
 nvfp4_status nvfp4_get_error(void* stream) {

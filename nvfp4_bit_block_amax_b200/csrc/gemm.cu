@@ -119,13 +119,14 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 }
 // Bounded wait: false when the limit ran out (the error word and the CTA's
 // abort flag are then set) or another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
         if (mbar_try(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort_flag = 1;
             atomicExch(&g_error_word, 1u);
             return false;
@@ -282,7 +283,30 @@ struct KParams {
     int64_t ldc;
     int tiles_m, tiles_n;
     int group_m;   // tile rasterization: groups of group_m M-tiles, M fastest inside a group
+    unsigned int* c_amax;   // nullable: atomic max of |C| (binary32 bits of the stored values)
 };
+
+// Fold this thread's maximum |C| (binary32 bits, non-negative) into c_amax:
+// one atomic per warp, once per kernel (the epilogue roles keep a running
+// maximum over all the tiles they drain).
+__device__ __forceinline__ void amax_publish(unsigned int* c_amax, uint32_t m) {
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if ((threadIdx.x & 31) == 0 && m) atomicMax(c_amax, m);
+}
+// Largest |bf16| among the packed pairs of one epilogue row: columns at or
+// past ncols (and rows at or past M) do not count.
+__device__ __forceinline__ uint32_t packed_row_amax(const uint32_t (&packed)[64], int ncols, bool row_ok) {
+    uint32_t acc = 0;
+    if (row_ok) {
+#pragma unroll
+        for (int g = 0; g < 64; ++g) {
+            uint32_t w = packed[g];
+            if (2 * g + 1 >= ncols) w = (2 * g < ncols) ? (w & 0xFFFFu) : 0u;
+            acc = absmax2(acc, w);
+        }
+    }
+    return absmax2_fold(acc);
+}
 
 // Tile t -> (tm, tn).  Tiles are taken in groups of group_m M-tiles; inside a
 // group M runs fastest, then N.  The CTAs working at the same time then share
@@ -303,7 +327,7 @@ __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& tm, in
 // bounded wait for the accumulator ran out.
 __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int half, int q, int lane, uint32_t tmem,
                                               float alpha, uint32_t bar_tfull, uint32_t bar_tempty,
-                                              uint32_t& acc_phase, volatile int* abort_flag) {
+                                              uint32_t& acc_phase, volatile int* abort_flag, uint32_t& amax_acc) {
     if (!mbar_wait(bar_tfull, acc_phase, abort_flag)) return false;
     tc_fence_after();
     int tm, tn;
@@ -337,6 +361,7 @@ __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int ha
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_tempty);
         acc_phase ^= 1;
+        if (p.c_amax) amax_acc = max(amax_acc, packed_row_amax(packed, ncols, row < p.M));
         if (row < p.M && ncols > 0) {
             __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + col0;
             if (ncols >= 128) {
@@ -354,6 +379,7 @@ __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int ha
         }
     } else {
         float* crow = reinterpret_cast<float*>(p.c) + (int64_t)row * p.ldc + col0;
+        float fmax = 0.0f;
 #pragma unroll 1
         for (int i = 0; i < 4; ++i) {
             uint32_t v[32];
@@ -369,14 +395,19 @@ __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int ha
                                                  __fmul_rn(__uint_as_float(v[4 * g + 3]), alpha));
                     if (cc + 4 <= ncols) {
                         *reinterpret_cast<float4*>(crow + cc) = f;
+                        fmax = fmaxf(fmaxf(fmaxf(fmax, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
                     } else {
                         const float ff[4] = {f.x, f.y, f.z, f.w};
                         for (int e = 0; e < 4; ++e)
-                            if (cc + e < ncols) crow[cc + e] = ff[e];
+                            if (cc + e < ncols) {
+                                crow[cc + e] = ff[e];
+                                fmax = fmaxf(fmax, fabsf(ff[e]));
+                            }
                     }
                 }
             }
         }
+        amax_acc = max(amax_acc, __float_as_uint(fmax));
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_tempty);
@@ -516,9 +547,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
         int prev_tile = -1;
+        uint32_t amax_acc = 0;   // max |C| of this thread's drained rows (binary32 bits)
 
         auto epilogue = [&](int tile) -> bool {
-            return epilogue_half(p, tile, 0, q, lane, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag);
+            return epilogue_half(p, tile, 0, q, lane, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag, amax_acc);
         };
 
         for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -581,13 +613,19 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             if (ok) prev_tile = tile;
         }
         if (ok && prev_tile >= 0) epilogue(prev_tile);
+        __syncwarp();
+        if (p.c_amax) amax_publish(p.c_amax, amax_acc);
     } else {
         // ---------------------------------------- epilogue, columns 128..255 ----
         const int q = warp & 3;
         const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
         uint32_t acc_phase = 0;
+        uint32_t amax_acc = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x)
-            if (!epilogue_half(p, tile, 1, q, lane, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag)) break;
+            if (!epilogue_half(p, tile, 1, q, lane, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag,
+                               amax_acc)) break;
+        __syncwarp();
+        if (p.c_amax) amax_publish(p.c_amax, amax_acc);
     }
 
     tc_fence_before();
@@ -626,7 +664,7 @@ constexpr uint32_t kIdescPair = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) <
 
 __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, int half, int q, int lane, uint32_t rank,
                                                    uint32_t tmem, float alpha, uint32_t bar_tfull, uint32_t bar_tempty,
-                                                   uint32_t& acc_phase, volatile int* abort_flag) {
+                                                   uint32_t& acc_phase, volatile int* abort_flag, uint32_t& amax_acc) {
     if (!mbar_wait_cluster(bar_tfull, acc_phase, abort_flag)) return false;
     tc_fence_after();
     int tm, tn;
@@ -663,6 +701,7 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
             }
         }
         release();
+        if (p.c_amax) amax_acc = max(amax_acc, packed_row_amax(packed, ncols, row < p.M));
         if (row < p.M && ncols > 0) {
             __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + col0;
             if (ncols >= 128) {
@@ -680,6 +719,7 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
         }
     } else {
         float* crow = reinterpret_cast<float*>(p.c) + (int64_t)row * p.ldc + col0;
+        float fmax = 0.0f;
 #pragma unroll 1
         for (int i = 0; i < 4; ++i) {
             uint32_t v[32];
@@ -695,14 +735,19 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
                                                  __fmul_rn(__uint_as_float(v[4 * g + 3]), alpha));
                     if (cc + 4 <= ncols) {
                         *reinterpret_cast<float4*>(crow + cc) = f;
+                        fmax = fmaxf(fmaxf(fmaxf(fmax, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
                     } else {
                         const float ff[4] = {f.x, f.y, f.z, f.w};
                         for (int e = 0; e < 4; ++e)
-                            if (cc + e < ncols) crow[cc + e] = ff[e];
+                            if (cc + e < ncols) {
+                                crow[cc + e] = ff[e];
+                                fmax = fmaxf(fmax, fabsf(ff[e]));
+                            }
                     }
                 }
             }
         }
+        amax_acc = max(amax_acc, __float_as_uint(fmax));
         release();
     }
     return true;
@@ -839,6 +884,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
         int prev_tile = -1;
+        uint32_t amax_acc = 0;   // max |C| of this thread's drained rows (binary32 bits)
         for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
             for (int kb = 0; kb < k_blocks; ++kb) {
                 // As in the single-SM kernel: wait for the stage, draining the
@@ -848,7 +894,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                     while (true) {
                         if (prev_tile >= 0 && mbar_test_cluster(bar_tfull, acc_phase)) {
                             if (!epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty,
-                                                    acc_phase, abort_flag)) { ok = false; break; }
+                                                    acc_phase, abort_flag, amax_acc)) { ok = false; break; }
                             prev_tile = -1;
                         }
                         if (mbar_test_cluster(bar_full + 8 * s, phase)) break;
@@ -895,21 +941,27 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
             }
             if (ok && prev_tile >= 0) {
                 if (!epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase,
-                                        abort_flag)) ok = false;
+                                        abort_flag, amax_acc)) ok = false;
                 prev_tile = -1;
             }
             if (ok) prev_tile = tile;
         }
         if (ok && prev_tile >= 0)
-            epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag);
+            epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag,
+                               amax_acc);
+        __syncwarp();
+        if (p.c_amax) amax_publish(p.c_amax, amax_acc);
     } else {
         // ---------------------------------------- epilogue, columns 128..255 ----
         const int q = warp & 3;
         const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
         uint32_t acc_phase = 0;
+        uint32_t amax_acc = 0;
         for (int tile = cluster; tile < num_tiles; tile += n_clusters)
             if (!epilogue_half_pair(p, tile, 1, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase,
-                                    abort_flag)) break;
+                                    abort_flag, amax_acc)) break;
+        __syncwarp();
+        if (p.c_amax) amax_publish(p.c_amax, amax_acc);
     }
 
     tc_fence_before();
@@ -919,6 +971,22 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS));
     }
+}
+
+// ------------------------------------------------------- wait self-test ----
+// The failure path of every bounded wait, exercised without a fault: one
+// thread waits on a barrier that nothing arrives on, with the caller's limit;
+// when it runs out the kernel raises the device error word and returns.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(smem_u32(&bar), 0, &abort_flag, limit_ns);
 }
 
 // ----------------------------------------------------------- host side -----
@@ -1017,6 +1085,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     p.out_bf16 = g.out_bf16;
     p.c = g.c;
     p.ldc = g.ldc;
+    p.c_amax = reinterpret_cast<unsigned int*>(g.c_amax);
     p.tiles_n = (int)ceil_div(g.N, BN);
     // The CTA-pair kernel is the default: per SM it moves 38 KB instead of
     // 54 KB from L2 per 256-wide K block.  NVFP4_GEMM_PAIR=0 selects the
@@ -1065,6 +1134,11 @@ unsigned int read_and_clear_error_word(cudaStream_t s, cudaError_t* err) {
     const unsigned int zero = 0;
     *err = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
     return w;
+}
+
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s) {
+    wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns);
+    return cudaGetLastError();
 }
 
 }  // namespace nvfp4

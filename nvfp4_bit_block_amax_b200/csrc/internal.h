@@ -24,6 +24,7 @@ struct QuantArgs {
     uint8_t* scales_mma;          // MMA layout or nullptr
     float* global_scale;
     uint32_t* partials;           // workspace
+    const float* given_amax;      // non-null: the tensor amax is known, skip the amax pass
 };
 
 struct Quant2dArgs {
@@ -36,6 +37,7 @@ struct Quant2dArgs {
     uint8_t* scales_mma_col;      // nullable
     float* global_scale;
     uint32_t* partials;
+    const float* given_amax;      // non-null: the tensor amax is known, skip the amax pass
 };
 
 cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches);
@@ -58,10 +60,12 @@ struct GemmArgs {
     int out_bf16;
     void* c;
     int64_t ldc;
+    float* c_amax;                // non-null: also max |C| over the stored values (zeroed by the caller)
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
 unsigned int read_and_clear_error_word(cudaStream_t s, cudaError_t* err);
+cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s);
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t mma_chunks_k(int64_t k) { return ceil_div(k / 16, 4); }

@@ -678,11 +678,15 @@ int launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
 }
 
 template <bool RHT, bool SR>
-cudaError_t run_rows(Params p, cudaStream_t s, int* launches) {
+cudaError_t run_rows(Params p, const float* given, cudaStream_t s, int* launches) {
     const int64_t units = p.rows * ((p.cols + 511) >> 9);
     const int64_t warps_needed = (units + 1) / 2;
     const int g = grid_for(rows_kernel<RHT, SR, false>, (warps_needed + 7) / 8);
-    if (RHT) {
+    if (given) {   // the tensor amax is known: it is the single partial
+        p.partials = const_cast<uint32_t*>(reinterpret_cast<const uint32_t*>(given));
+        p.n_partials = 1;
+        *launches -= 1;
+    } else if (RHT) {
         p.n_partials = g;
         rows_kernel<true, false, true><<<g, kThreads, 0, s>>>(p);
     } else {
@@ -694,10 +698,14 @@ cudaError_t run_rows(Params p, cudaStream_t s, int* launches) {
 }
 
 template <bool RHT, bool SR>
-cudaError_t run_cols(Params p, cudaStream_t s, int* launches) {
+cudaError_t run_cols(Params p, const float* given, cudaStream_t s, int* launches) {
     const int64_t tiles = ((p.rows + 127) >> 7) * ((p.cols + 255) >> 8);
     const int g = grid_for(cols_kernel<RHT, SR, false>, tiles);
-    if (RHT) {
+    if (given) {
+        p.partials = const_cast<uint32_t*>(reinterpret_cast<const uint32_t*>(given));
+        p.n_partials = 1;
+        *launches -= 1;
+    } else if (RHT) {
         p.n_partials = g;
         cols_kernel<true, false, true><<<g, kThreads, 0, s>>>(p);
     } else {
@@ -733,12 +741,13 @@ cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches
         if (e != cudaSuccess) return e;
     }
     const bool sr = a.rounding == 1;
+    const float* g = a.given_amax;
     if (!a.transpose) {
-        if (a.rht) return sr ? run_rows<true, true>(p, s, launches) : run_rows<true, false>(p, s, launches);
-        return sr ? run_rows<false, true>(p, s, launches) : run_rows<false, false>(p, s, launches);
+        if (a.rht) return sr ? run_rows<true, true>(p, g, s, launches) : run_rows<true, false>(p, g, s, launches);
+        return sr ? run_rows<false, true>(p, g, s, launches) : run_rows<false, false>(p, g, s, launches);
     }
-    if (a.rht) return sr ? run_cols<true, true>(p, s, launches) : run_cols<true, false>(p, s, launches);
-    return sr ? run_cols<false, true>(p, s, launches) : run_cols<false, false>(p, s, launches);
+    if (a.rht) return sr ? run_cols<true, true>(p, g, s, launches) : run_cols<true, false>(p, g, s, launches);
+    return sr ? run_cols<false, true>(p, g, s, launches) : run_cols<false, false>(p, g, s, launches);
 }
 
 cudaError_t launch_quantize_2d(const Quant2dArgs& a, cudaStream_t s, int* launches) {
@@ -766,7 +775,13 @@ cudaError_t launch_quantize_2d(const Quant2dArgs& a, cudaStream_t s, int* launch
     }
     const int64_t tiles = ((a.rows + 127) >> 7) * ((a.cols + 255) >> 8);
     const int g = a.codes_col ? grid_for(q2d_kernel<true>, tiles) : grid_for(q2d_kernel<false>, tiles);
-    p.n_partials = launch_amax_plain(a.w, a.rows, a.cols, a.ld, a.partials, s);
+    if (a.given_amax) {   // the tensor amax is known: it is the single partial
+        p.partials = const_cast<uint32_t*>(reinterpret_cast<const uint32_t*>(a.given_amax));
+        p.n_partials = 1;
+        *launches -= 1;
+    } else {
+        p.n_partials = launch_amax_plain(a.w, a.rows, a.cols, a.ld, a.partials, s);
+    }
     if (a.codes_col) q2d_kernel<true><<<g, kThreads, 0, s>>>(p);
     else q2d_kernel<false><<<g, kThreads, 0, s>>>(p);
     *launches += 2;
@@ -841,6 +856,7 @@ cudaError_t launch_quantize_1d_noalloc(const QuantArgs& a, cudaStream_t s, int* 
     }
     QuantArgs b = a;
     b.rht = 0;
+    b.given_amax = nullptr;
     b.partials = scratch;
     return launch_quantize_1d(b, s, launches);
 }

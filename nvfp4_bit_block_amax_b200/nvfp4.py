@@ -22,6 +22,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 
 NVFP4_OK = 0
+(NVFP4_ERR_INVALID_ARG, NVFP4_ERR_UNSUPPORTED_SHAPE, NVFP4_ERR_MISALIGNED, NVFP4_ERR_CUDA, NVFP4_ERR_TIMEOUT,
+ NVFP4_ERR_WORKSPACE) = 1, 2, 3, 4, 5, 6
 NVFP4_RNE, NVFP4_SR = 0, 1
 NVFP4_SCALE_1D, NVFP4_SCALE_2D = 0, 1
 NVFP4_OUT_F32, NVFP4_OUT_BF16 = 0, 1
@@ -30,6 +32,8 @@ EXPORTS = (
     "nvfp4_version", "nvfp4_status_string", "nvfp4_workspace_size", "nvfp4_mma_scale_bytes",
     "nvfp4_quantize_1d", "nvfp4_rht_quantize_sr", "nvfp4_quantize_2d", "nvfp4_dequantize", "nvfp4_gemm",
     "nvfp4_scales_to_mma", "nvfp4_kernel_launches", "nvfp4_get_error", "nvfp4_quantize_1d_noalloc",
+    "nvfp4_selftest_wait_timeout", "nvfp4_quantize_1d_from_amax", "nvfp4_quantize_2d_from_amax",
+    "nvfp4_gemm_amax",
 )
 
 _lib = None
@@ -76,6 +80,14 @@ def lib():
         L.nvfp4_kernel_launches.argtypes = []
         L.nvfp4_get_error.restype = ci
         L.nvfp4_get_error.argtypes = [vp]
+        L.nvfp4_selftest_wait_timeout.restype = ci
+        L.nvfp4_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp]
+        L.nvfp4_quantize_1d_from_amax.restype = ci
+        L.nvfp4_quantize_1d_from_amax.argtypes = [vp, i64, i64, i64, ci, ci, u64, vp, vp, vp, vp, vp, vp]
+        L.nvfp4_quantize_2d_from_amax.restype = ci
+        L.nvfp4_quantize_2d_from_amax.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.nvfp4_gemm_amax.restype = ci
+        L.nvfp4_gemm_amax.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, i64, vp, vp]
         _lib = L
     return _lib
 
@@ -165,6 +177,27 @@ def nvfp4_gemm(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K
         _p(c), ldc, _stream(stream)))
 
 
+def nvfp4_gemm_amax(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K, out_dtype, c, ldc, c_amax,
+                    stream=None):
+    _check("nvfp4_gemm_amax", lib().nvfp4_gemm_amax(
+        _p(a_codes), _p(a_scales_mma), _p(a_gs), _p(b_codes), _p(b_scales_mma), _p(b_gs), M, N, K, out_dtype,
+        _p(c), ldc, _p(c_amax), _stream(stream)))
+
+
+def nvfp4_quantize_1d_from_amax(x, rows, cols, ld, transpose, rounding, sr_seed, amax, codes, scales, scales_mma,
+                                global_scale, stream=None):
+    _check("nvfp4_quantize_1d_from_amax", lib().nvfp4_quantize_1d_from_amax(
+        _p(x), rows, cols, ld, transpose, rounding, sr_seed, _p(amax), _p(codes), _p(scales), _p(scales_mma),
+        _p(global_scale), _stream(stream)))
+
+
+def nvfp4_quantize_2d_from_amax(w, rows, cols, ld, amax, codes_row, codes_col, scales, scales_mma_row,
+                                scales_mma_col, global_scale, stream=None):
+    _check("nvfp4_quantize_2d_from_amax", lib().nvfp4_quantize_2d_from_amax(
+        _p(w), rows, cols, ld, _p(amax), _p(codes_row), _p(codes_col), _p(scales), _p(scales_mma_row),
+        _p(scales_mma_col), _p(global_scale), _stream(stream)))
+
+
 def nvfp4_scales_to_mma(scales, scale_mode, rows, k, scales_mma, stream=None):
     _check("nvfp4_scales_to_mma", lib().nvfp4_scales_to_mma(
         _p(scales), scale_mode, rows, k, _p(scales_mma), _stream(stream)))
@@ -172,6 +205,10 @@ def nvfp4_scales_to_mma(scales, scale_mode, rows, k, scales_mma, stream=None):
 
 def nvfp4_get_error(stream=None) -> int:
     return lib().nvfp4_get_error(_stream(stream))
+
+
+def nvfp4_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    return lib().nvfp4_selftest_wait_timeout(int(limit_ns), _stream(stream))
 
 
 # --------------------------------------------------------- torch helpers ----
@@ -209,8 +246,9 @@ def _empty_u8(n, device):
 
 def quantize_1d(x: torch.Tensor, transpose: bool = False, rounding: int = NVFP4_RNE, sr_seed: int = 0,
                 rht: bool = False, rht_seed: int = 0, plain_scales: bool = True, mma_scales: bool = True,
-                stream=None) -> Quantized:
-    """Quantize a bf16 [rows x cols] tensor (or its transpose) with 16-element blocks."""
+                stream=None, amax: Optional[torch.Tensor] = None) -> Quantized:
+    """Quantize a bf16 [rows x cols] tensor (or its transpose) with 16-element blocks.
+    With `amax` (a device float holding max |x|) the amax pass is skipped."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     rows, cols = x.shape
     qr, qc = (cols, rows) if transpose else (rows, cols)
@@ -220,7 +258,11 @@ def quantize_1d(x: torch.Tensor, transpose: bool = False, rounding: int = NVFP4_
     smma = _empty_u8(nvfp4_mma_scale_bytes(qr, qc), dev) if mma_scales else None
     gs = torch.empty(1, dtype=torch.float32, device=dev)
     ws = workspace(dev)
-    if rht:
+    if amax is not None:
+        assert not rht, "the amax of the rotated tensor is not known to a producer"
+        nvfp4_quantize_1d_from_amax(x, rows, cols, x.stride(0), int(transpose), rounding, sr_seed, amax, codes,
+                                    scales, smma, gs, stream)
+    elif rht:
         nvfp4_rht_quantize_sr(x, rows, cols, x.stride(0), int(transpose), rht_seed, rounding, sr_seed, codes,
                               scales, smma, gs, ws, ws.numel(), stream)
     else:
@@ -230,7 +272,7 @@ def quantize_1d(x: torch.Tensor, transpose: bool = False, rounding: int = NVFP4_
 
 
 def quantize_2d(w: torch.Tensor, columnwise: bool = True, plain_scales: bool = True, mma_scales: bool = True,
-                stream=None) -> Quantized:
+                stream=None, amax: Optional[torch.Tensor] = None) -> Quantized:
     """Quantize a bf16 weight with 16x16 tiles (rowwise codes, optional columnwise copy)."""
     assert w.dtype == torch.bfloat16 and w.dim() == 2 and w.stride(1) == 1
     rows, cols = w.shape
@@ -242,7 +284,10 @@ def quantize_2d(w: torch.Tensor, columnwise: bool = True, plain_scales: bool = T
     mc = _empty_u8(nvfp4_mma_scale_bytes(cols, rows), dev) if (mma_scales and columnwise) else None
     gs = torch.empty(1, dtype=torch.float32, device=dev)
     ws = workspace(dev)
-    nvfp4_quantize_2d(w, rows, cols, w.stride(0), cr, cc, sc, mr, mc, gs, ws, ws.numel(), stream)
+    if amax is not None:
+        nvfp4_quantize_2d_from_amax(w, rows, cols, w.stride(0), amax, cr, cc, sc, mr, mc, gs, stream)
+    else:
+        nvfp4_quantize_2d(w, rows, cols, w.stride(0), cr, cc, sc, mr, mc, gs, ws, ws.numel(), stream)
     return Quantized(cr, sc, mr, gs, rows, cols, codes_col=cc, scales_mma_col=mc)
 
 
@@ -255,12 +300,18 @@ def dequantize(q: Quantized, scale_mode: int = NVFP4_SCALE_1D, out_dtype: int = 
 
 
 def gemm(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M: int, N: int, K: int,
-         out_dtype: int = NVFP4_OUT_BF16, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """C = alpha * A . B^T with NVFP4 operands (MMA-layout scales)."""
+         out_dtype: int = NVFP4_OUT_BF16, out: Optional[torch.Tensor] = None, stream=None,
+         amax_out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """C = alpha * A . B^T with NVFP4 operands (MMA-layout scales).  With
+    `amax_out` (a device float) the epilogue also writes max |C| there."""
     if out is None:
         dt = torch.float32 if out_dtype == NVFP4_OUT_F32 else torch.bfloat16
         ldc = (N + 7) // 8 * 8
         out = torch.empty(M, ldc, dtype=dt, device=a_codes.device)[:, :N]
-    nvfp4_gemm(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K, out_dtype, out,
-               out.stride(0), stream)
+    if amax_out is not None:
+        nvfp4_gemm_amax(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K, out_dtype, out,
+                        out.stride(0), amax_out, stream)
+    else:
+        nvfp4_gemm(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K, out_dtype, out,
+                   out.stride(0), stream)
     return out

@@ -113,3 +113,11 @@ def test_missing_library_raises(monkeypatch, tmp_path):
     monkeypatch.setattr(N, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(OSError):
         N.lib()
+
+
+def test_python_constants_match_header_enums():
+    """The binding's status / mode constants carry the header's values."""
+    import re
+    hdr = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
+    for name, value in re.findall(r"\b(NVFP4_[A-Z0-9_]+) = (\d+)", hdr):
+        assert getattr(N, name) == int(value), name
