@@ -398,3 +398,65 @@ void nvfp4o_e2m1_sr_batch(const float* v, int64_t n, uint64_t seed, uint64_t fir
 void nvfp4o_e4m3_batch(const float* s, int64_t n, uint8_t* codes) {
     for (int64_t i = 0; i < n; ++i) codes[i] = (uint8_t)nvfp4o_e4m3_rne_satfinite(s[i]);
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4 [P2 "MXFP4:开放标准,但精度较粗" -- 32 values share one scale that can
+ * only be a power of two, stored as E8M0; P5 "Generic FP4, MXFP4, and NVFP4"
+ * -- E2M1 payloads, one E8M0 scale per 32 values, no tensor-level scale].
+ * The pages do not say how the power of two is chosen; reading: the OCP
+ * microscaling rule the format is named after -- X = 2^(floor(log2(amax)) -
+ * 2), 2 being the exponent of the largest E2M1 value (6 = 1.5 * 2^2), so the
+ * block maximum lands in [4, 8) and values above 6 saturate.  The exponent is
+ * clamped to the E8M0 range [-127, 127]; an all-zero block gets -127.
+ * E8M0 code = exponent + 127 (255, NaN, is never produced). */
+int nvfp4o_mx_scale_exp(float block_amax) {
+    if (!(block_amax > 0.0f)) return -127;
+    int e2;
+    (void)frexp((double)block_amax, &e2);        /* amax = f * 2^e2, f in [0.5, 1) */
+    int e = (e2 - 1) - 2;                        /* floor(log2(amax)) - 2 */
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+double nvfp4o_e8m0_value(int code) { return ldexp(1.0, code - 127); }
+
+/* One element: v = x / 2^e (exact in double), E2M1 by nearest-even with
+ * saturation at +-6, sign kept. */
+int nvfp4o_mx_encode_element(float x, int e) {
+    double v = ldexp((double)x, -e);
+    int sign = signbit(x) ? 8 : 0;
+    return sign | e2m1_mag_rne(fabs(v));
+}
+
+/* MXFP4 quantization of bf16 x [rows x cols] (cols % 32 == 0), blocks of 32
+ * along each row: codes [rows x cols/2], scales (E8M0 codes) [rows x cols/32]. */
+void nvfp4o_mx_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
+                        uint8_t* scales) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t b = 0; b < cols / 32; ++b) {
+            float amax = 0.0f;
+            for (int j = 0; j < 32; ++j) {
+                float a = fabsf(bf16_to_float(x[r * ld + 32 * b + j]));
+                if (a > amax) amax = a;
+            }
+            int e = nvfp4o_mx_scale_exp(amax);
+            scales[r * (cols / 32) + b] = (uint8_t)(e + 127);
+            for (int j = 0; j < 32; j += 2) {
+                int lo = nvfp4o_mx_encode_element(bf16_to_float(x[r * ld + 32 * b + j]), e);
+                int hi = nvfp4o_mx_encode_element(bf16_to_float(x[r * ld + 32 * b + j + 1]), e);
+                codes[r * (cols / 2) + 16 * b + j / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+}
+
+/* Reconstruction x = value(code) * 2^e, in binary32 (exact unless it underflows). */
+void nvfp4o_mx_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols, float* out) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            uint8_t byte = codes[r * (cols / 2) + c / 2];
+            int code = (c & 1) ? (byte >> 4) : (byte & 0xF);
+            double s = nvfp4o_e8m0_value(scales[r * (cols / 32) + c / 32]);
+            out[r * cols + c] = (float)(nvfp4o_e2m1_value(code) * s);
+        }
+}

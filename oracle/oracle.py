@@ -86,6 +86,16 @@ def lib():
             L.nvfp4o_e4m3_batch.argtypes = [vp, i64, vp]
             L.nvfp4o_dequantize.restype = None
             L.nvfp4o_dequantize.argtypes = [vp, vp, ci, fp, i64, i64, vp]
+            L.nvfp4o_mx_scale_exp.restype = ci
+            L.nvfp4o_mx_scale_exp.argtypes = [fp]
+            L.nvfp4o_e8m0_value.restype = ctypes.c_double
+            L.nvfp4o_e8m0_value.argtypes = [ci]
+            L.nvfp4o_mx_encode_element.restype = ci
+            L.nvfp4o_mx_encode_element.argtypes = [fp, ci]
+            L.nvfp4o_mx_quantize.restype = None
+            L.nvfp4o_mx_quantize.argtypes = [vp, i64, i64, i64, vp, vp]
+            L.nvfp4o_mx_dequantize.restype = None
+            L.nvfp4o_mx_dequantize.argtypes = [vp, vp, i64, i64, vp]
             _lib = L
     return _lib
 
@@ -308,3 +318,45 @@ def gemm_reference(a_hat: np.ndarray, b_hat: np.ndarray):
     a = np.asarray(a_hat, dtype=np.float64)
     b = np.asarray(b_hat, dtype=np.float64)
     return a @ b.T, np.abs(a) @ np.abs(b).T
+
+
+# ------------------------------------------------------------------ MXFP4 ----
+def mx_scale_exp(block_amax: float) -> int:
+    """Exponent e of the block's power-of-two scale 2^e (E8M0 code e + 127):
+    floor(log2(amax)) - 2, clamped to [-127, 127]; -127 for an all-zero block
+    ("MXFP4 和 NVFP4 的区别", "MXFP4:开放标准,但精度较粗"; the OCP rule)."""
+    return lib().nvfp4o_mx_scale_exp(float(block_amax))
+
+
+def e8m0_value(code: int) -> float:
+    return lib().nvfp4o_e8m0_value(int(code))
+
+
+def mx_encode_element(x: float, e: int) -> int:
+    return lib().nvfp4o_mx_encode_element(float(x), int(e))
+
+
+def mx_quantize(x: np.ndarray):
+    """MXFP4 quantization of bf16 bits x [rows x cols] (cols % 32 == 0):
+    (codes [rows x cols/2], E8M0 scale codes [rows x cols/32])."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 32), dtype=np.uint8)
+    lib().nvfp4o_mx_quantize(_ptr(x), rows, cols, cols, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def mx_dequantize(codes: np.ndarray, scales: np.ndarray, rows: int, cols: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    out = np.zeros((rows, cols), dtype=np.float32)
+    lib().nvfp4o_mx_dequantize(_ptr(codes), _ptr(scales), rows, cols, _ptr(out))
+    return out
+
+
+def mx_gemm_reference(a_codes, a_scales, b_codes, b_scales, M: int, N: int, K: int):
+    """float64 C = A_hat . B_hat^T of two MXFP4 operands and S = |A_hat| . |B_hat|^T."""
+    a_hat = mx_dequantize(a_codes, a_scales, M, K).astype(np.float64)
+    b_hat = mx_dequantize(b_codes, b_scales, N, K).astype(np.float64)
+    return a_hat @ b_hat.T, np.abs(a_hat) @ np.abs(b_hat).T
