@@ -52,7 +52,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default=None,
                     choices=["gemm", "gemm_amax", "quantize_1d", "quantize_1d_sr", "quantize_2d", "rht_t_sr",
-                             "rht_t_rne", "quantize_1d_from_amax", "quantize_2d_from_amax",
+                             "rht_t_rne", "quantize_1d_from_amax", "quantize_2d_from_amax", "mx_quantize",
+                             "mx_gemm",
                              "dequantize"],
                     help="time one kernel family alone on --shape (profiling mode)")
     ap.add_argument("--shape", default=None, help="M,N,K for gemm; rows,cols otherwise")
@@ -480,7 +481,16 @@ def micro(args):
     g = torch.Generator(device=dev)
     g.manual_seed(1234)
     s = torch.cuda.Stream(device=dev)
-    if args.op in ("gemm", "gemm_amax"):
+    if args.op == "mx_gemm":
+        M, Nn, K = dims
+        a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        b = torch.randint(0, 256, (Nn, K // 2), dtype=torch.uint8, device=dev, generator=g)
+        sa = torch.randint(120, 130, (N.nvfp4_mma_scale_bytes(M, K),), dtype=torch.uint8, device=dev, generator=g)
+        sb = torch.randint(120, 130, (N.nvfp4_mma_scale_bytes(Nn, K),), dtype=torch.uint8, device=dev, generator=g)
+        c = torch.empty(M, Nn, dtype=torch.bfloat16, device=dev)
+        fn = lambda: N.nvfp4_mxfp4_gemm(a, sa, b, sb, M, Nn, K, N.NVFP4_OUT_BF16, c, Nn, s)
+        work, unit = 2.0 * M * Nn * K, "TFLOP/s"
+    elif args.op in ("gemm", "gemm_amax"):
         M, Nn, K = dims
         a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g)
         b = torch.randint(0, 256, (Nn, K // 2), dtype=torch.uint8, device=dev, generator=g)
@@ -519,6 +529,9 @@ def micro(args):
             sm2 = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)
             fn = lambda: N.nvfp4_quantize_2d_from_amax(x, R, C, C, amax, codes, cc, None, smma, sm2, gs, s)
             work = R * C * (2 + 0.5 + 0.5 + 2 / 16)
+        elif args.op == "mx_quantize":
+            fn = lambda: N.nvfp4_mxfp4_quantize(x, R, C, C, codes, None, smma, s)
+            work = R * C * (2 + 0.5 + 1 / 32)
         elif args.op == "quantize_2d":
             cc = torch.empty(C, R // 2, dtype=torch.uint8, device=dev)
             sm2 = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)

@@ -251,6 +251,40 @@ nvfp4_status nvfp4_gemm_amax(const uint8_t* a_codes, const uint8_t* a_scales_mma
 nvfp4_status nvfp4_scales_to_mma(const uint8_t* scales, int scale_mode, int64_t rows, int64_t k,
                                  uint8_t* scales_mma, void* stream);
 
+/* MXFP4 ["MXFP4 和 NVFP4 的区别", "MXFP4:开放标准,但精度较粗" -- 32 values
+ * share one scale restricted to powers of two, stored as E8M0; "NVFP4 Is a
+ * Scaling System, Not Just a 4-Bit Number", "Generic FP4, MXFP4, and NVFP4"
+ * -- E2M1 payloads, no tensor-level scale; "Melatih model dalam 4 bit",
+ * "Anatomi NVFP4" -- 4.25 bits per element].  The library's MXFP4 variant
+ * of the path, for comparison with NVFP4 on the same kernels.
+ *
+ * Quantize (RNE, one pass: no tensor amax is needed):
+ *   per 32-block along K, e = clamp(floor(log2(block amax)) - 2, -127, 127)
+ *   (-127 for an all-zero block), scale code = e + 127 (E8M0), element code =
+ *   E2M1 nearest-even of x / 2^e, saturating at +-6, sign kept.
+ *   x bf16 [rows x cols] (row stride ld); cols % 32 == 0.
+ *   codes [rows x cols/2]; scales [rows x cols/32] E8M0 codes (nullable);
+ *   scales_mma (nullable, one of the two required): the NVFP4 MMA layout of
+ *   nvfp4_mma_scale_bytes(rows, cols) bytes, in which the 4-byte entry of a
+ *   row and 64-wide K step holds the step's two E8M0 codes in bytes 0 and 1
+ *   and zeros in bytes 2 and 3. */
+nvfp4_status nvfp4_mxfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
+                                  uint8_t* scales, uint8_t* scales_mma, void* stream);
+
+/* MXFP4 reconstruction: out = RN(value(code) * 2^e) in binary32 (exact unless
+ * it underflows), NVFP4_OUT_BF16 then rounds to bf16.  codes [rows x cols/2],
+ * scales [rows x cols/32] (plain), out [rows x cols]; cols % 32 == 0. */
+nvfp4_status nvfp4_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                    int out_dtype, void* out, void* stream);
+
+/* MXFP4 GEMM, C = A . B^T with FP32 accumulation (no global scales, alpha 1):
+ * the NVFP4 GEMM kernels with tcgen05.mma block_scale.scale_vec::2X and UE8M0
+ * scales.  Operands as nvfp4_gemm (codes K-major, MMA-layout scales from
+ * nvfp4_mxfp4_quantize); same shape, alignment and output rules. */
+nvfp4_status nvfp4_mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales_mma, const uint8_t* b_codes,
+                              const uint8_t* b_scales_mma, int64_t M, int64_t N, int64_t K, int out_dtype, void* c,
+                              int64_t ldc, void* stream);
+
 /* Number of kernels (and memset nodes excluded) this library has enqueued in
  * this process; instrumentation for benchmarks. */
 long long nvfp4_kernel_launches(void);

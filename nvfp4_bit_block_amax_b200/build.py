@@ -25,6 +25,7 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler",
 UNITS = {
     "quant.cu": ["--fmad=false"],
     "gemm.cu": [],
+    "mxfp4.cu": [],
     "api.cu": [],
 }
 HEADERS = ["common.cuh", "internal.h"]

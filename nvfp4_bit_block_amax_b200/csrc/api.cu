@@ -220,15 +220,15 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int s
 static nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales_mma, const float* a_gs,
                               const uint8_t* b_codes, const uint8_t* b_scales_mma, const float* b_gs, int64_t M,
                               int64_t N, int64_t K, int out_dtype, void* c, int64_t ldc, float* c_amax,
-                              void* stream) {
-    if (!a_codes || !a_scales_mma || !a_gs || !b_codes || !b_scales_mma || !b_gs || !c)
-        return NVFP4_ERR_INVALID_ARG;
+                              void* stream, int mx = 0) {
+    if (!a_codes || !a_scales_mma || !b_codes || !b_scales_mma || !c) return NVFP4_ERR_INVALID_ARG;
+    if (!mx && (!a_gs || !b_gs)) return NVFP4_ERR_INVALID_ARG;
     if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
     if (M < 1 || N < 1 || K < 1 || ldc < N || M >= kMaxDim || N >= kMaxDim || K >= kMaxDim)
         return NVFP4_ERR_INVALID_ARG;
     if (K % 64) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales_mma) || !aligned16(b_scales_mma) ||
-        !aligned16(c) || ldc % 8 || !aligned4(a_gs) || !aligned4(b_gs))
+        !aligned16(c) || ldc % 8 || (!mx && (!aligned4(a_gs) || !aligned4(b_gs))))
         return NVFP4_ERR_MISALIGNED;
     GemmArgs g{};
     g.a = a_codes;
@@ -244,6 +244,7 @@ static nvfp4_status gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales_mm
     g.c = c;
     g.ldc = ldc;
     g.c_amax = c_amax;
+    g.mx = mx;
     if (c_amax) {
         cudaError_t z = cudaMemsetAsync(c_amax, 0, sizeof(float), static_cast<cudaStream_t>(stream));
         if (z != cudaSuccess) return NVFP4_ERR_CUDA;
@@ -268,6 +269,39 @@ nvfp4_status nvfp4_gemm_amax(const uint8_t* a_codes, const uint8_t* a_scales_mma
     if (!aligned4(c_amax)) return NVFP4_ERR_MISALIGNED;
     return gemm_impl(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K, out_dtype, c, ldc, c_amax,
                      stream);
+}
+
+nvfp4_status nvfp4_mxfp4_quantize(const void* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
+                                  uint8_t* scales, uint8_t* scales_mma, void* stream) {
+    if (!x || !codes || (!scales && !scales_mma)) return NVFP4_ERR_INVALID_ARG;
+    if (rows < 1 || cols < 1 || ld < cols || rows >= kMaxDim || cols >= kMaxDim) return NVFP4_ERR_INVALID_ARG;
+    if (cols % 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld % 8 || !aligned16(x) || !aligned16(codes) || (scales_mma && !aligned16(scales_mma)))
+        return NVFP4_ERR_MISALIGNED;
+    cudaError_t e = launch_mx_quantize(static_cast<const uint16_t*>(x), rows, cols, ld, codes, scales, scales_mma,
+                                       static_cast<cudaStream_t>(stream));
+    g_launches += 1;
+    return from_cuda(e);
+}
+
+nvfp4_status nvfp4_mxfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                    int out_dtype, void* out, void* stream) {
+    if (!codes || !scales || !out) return NVFP4_ERR_INVALID_ARG;
+    if (out_dtype != NVFP4_OUT_F32 && out_dtype != NVFP4_OUT_BF16) return NVFP4_ERR_INVALID_ARG;
+    if (rows < 1 || cols < 1 || rows >= kMaxDim || cols >= kMaxDim) return NVFP4_ERR_INVALID_ARG;
+    if (cols % 32) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(codes) || !aligned16(out)) return NVFP4_ERR_MISALIGNED;
+    cudaError_t e = launch_mx_dequantize(codes, scales, rows, cols, out_dtype == NVFP4_OUT_BF16, out,
+                                         static_cast<cudaStream_t>(stream));
+    g_launches += 1;
+    return from_cuda(e);
+}
+
+nvfp4_status nvfp4_mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales_mma, const uint8_t* b_codes,
+                              const uint8_t* b_scales_mma, int64_t M, int64_t N, int64_t K, int out_dtype, void* c,
+                              int64_t ldc, void* stream) {
+    return gemm_impl(a_codes, a_scales_mma, nullptr, b_codes, b_scales_mma, nullptr, M, N, K, out_dtype, c, ldc,
+                     nullptr, stream, 1);
 }
 
 nvfp4_status nvfp4_scales_to_mma(const uint8_t* scales, int scale_mode, int64_t rows, int64_t k,

@@ -149,14 +149,25 @@ __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence:
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
+// NVFP4: one UE4M3 scale per 16 elements (scale_vec::4X).  MXFP4: one UE8M0
+// scale per 32 elements (scale_vec::2X), in bytes 0-1 of the same 4-byte
+// scale entry per row and 64-wide K step.
 __device__ __forceinline__ void tc_mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
-        ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
-        : "memory");
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate, bool mx) {
+    if (mx)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+            : "memory");
 }
 __device__ __forceinline__ void tc_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -251,13 +262,21 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
         : "memory");
 }
 __device__ __forceinline__ void tc_mma_nvf4_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                                 uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
-        ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
-        : "memory");
+                                                 uint32_t sfa, uint32_t sfb, uint32_t accumulate, bool mx) {
+    if (mx)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+            : "memory");
 }
 
 // Shared-memory matrix descriptor: K-major operand tile of rows x 128 bytes,
@@ -270,6 +289,7 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
 // Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
 // UE4M3 scales, dense K = 64, M = 128, N = 256.
 constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+constexpr uint32_t kIdescUe8m0 = 1u << 23;   // scale type UE8M0 (MXFP4) instead of UE4M3
 
 struct KParams {
     const uint8_t* sfa;
@@ -284,6 +304,7 @@ struct KParams {
     int tiles_m, tiles_n;
     int group_m;   // tile rasterization: groups of group_m M-tiles, M fastest inside a group
     unsigned int* c_amax;   // nullable: atomic max of |C| (binary32 bits of the stored values)
+    int mx;                 // MXFP4 operands: UE8M0 scales per 32 elements, no global scales (alpha = 1)
 };
 
 // Fold this thread's maximum |C| (binary32 bits, non-negative) into c_amax:
@@ -506,6 +527,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             int s = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
+            const uint32_t idesc = kIdesc | (p.mx ? kIdescUe8m0 : 0u);
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 if (!mbar_wait(bar_tempty, acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
@@ -520,8 +542,8 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     const uint32_t sfa_col = tmem + SF_COL + s * 48;
                     const uint32_t sfb_col = sfa_col + 16;
                     for (int j = 0; j < nk; ++j)
-                        tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32), kIdesc,
-                                    sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
+                        tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32), idesc,
+                                    sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0, p.mx);
                     tc_commit(bar_empty + 8 * s);
                     if (++s == STAGES) { s = 0; phase ^= 1; }
                 }
@@ -542,7 +564,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         // the 16 bytes at offset 16 l of the step's 512-byte scale chunks.
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
+        const float alpha = p.a_gs ? __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs)) : 1.0f;
         int s = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
@@ -618,7 +640,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     } else {
         // ---------------------------------------- epilogue, columns 128..255 ----
         const int q = warp & 3;
-        const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
+        const float alpha = p.a_gs ? __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs)) : 1.0f;
         uint32_t acc_phase = 0;
         uint32_t amax_acc = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x)
@@ -843,6 +865,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
             int s = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
+            const uint32_t idesc = kIdescPair | (p.mx ? kIdescUe8m0 : 0u);
             for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
                 if (!mbar_wait_cluster(bar_tempty, acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
@@ -858,7 +881,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                     const uint32_t sfb_col = sfa_col + 16;
                     for (int j = 0; j < nk; ++j)
                         tc_mma_nvf4_pair(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32),
-                                         kIdescPair, sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0);
+                                         idesc, sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0, p.mx);
                     tc_commit_pair(bar_empty + 8 * s);
                     if (++s == P_STAGES) { s = 0; phase ^= 1; }
                 }
@@ -879,7 +902,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
         // ------------------------------- scales -> TMEM, and the epilogue ----
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
+        const float alpha = p.a_gs ? __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs)) : 1.0f;
         int s = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
@@ -954,7 +977,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     } else {
         // ---------------------------------------- epilogue, columns 128..255 ----
         const int q = warp & 3;
-        const float alpha = __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs));
+        const float alpha = p.a_gs ? __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs)) : 1.0f;
         uint32_t acc_phase = 0;
         uint32_t amax_acc = 0;
         for (int tile = cluster; tile < num_tiles; tile += n_clusters)
@@ -1086,6 +1109,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     p.c = g.c;
     p.ldc = g.ldc;
     p.c_amax = reinterpret_cast<unsigned int*>(g.c_amax);
+    p.mx = g.mx;
     p.tiles_n = (int)ceil_div(g.N, BN);
     // The CTA-pair kernel is the default: per SM it moves 38 KB instead of
     // 54 KB from L2 per 256-wide K block.  NVFP4_GEMM_PAIR=0 selects the

@@ -61,11 +61,16 @@ struct GemmArgs {
     void* c;
     int64_t ldc;
     float* c_amax;                // non-null: also max |C| over the stored values (zeroed by the caller)
+    int mx;                       // MXFP4 operands (UE8M0 per 32, a_gs = b_gs = nullptr, alpha = 1)
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
 unsigned int read_and_clear_error_word(cudaStream_t s, cudaError_t* err);
 cudaError_t launch_wait_selftest(unsigned long long limit_ns, cudaStream_t s);
+cudaError_t launch_mx_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes,
+                               uint8_t* scales, uint8_t* scales_mma, cudaStream_t s);
+cudaError_t launch_mx_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                                 int out_bf16, void* out, cudaStream_t s);
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline int64_t mma_chunks_k(int64_t k) { return ceil_div(k / 16, 4); }

@@ -33,7 +33,7 @@ EXPORTS = (
     "nvfp4_quantize_1d", "nvfp4_rht_quantize_sr", "nvfp4_quantize_2d", "nvfp4_dequantize", "nvfp4_gemm",
     "nvfp4_scales_to_mma", "nvfp4_kernel_launches", "nvfp4_get_error", "nvfp4_quantize_1d_noalloc",
     "nvfp4_selftest_wait_timeout", "nvfp4_quantize_1d_from_amax", "nvfp4_quantize_2d_from_amax",
-    "nvfp4_gemm_amax",
+    "nvfp4_gemm_amax", "nvfp4_mxfp4_quantize", "nvfp4_mxfp4_dequantize", "nvfp4_mxfp4_gemm",
 )
 
 _lib = None
@@ -88,6 +88,12 @@ def lib():
         L.nvfp4_quantize_2d_from_amax.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
         L.nvfp4_gemm_amax.restype = ci
         L.nvfp4_gemm_amax.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, vp, i64, vp, vp]
+        L.nvfp4_mxfp4_quantize.restype = ci
+        L.nvfp4_mxfp4_quantize.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
+        L.nvfp4_mxfp4_dequantize.restype = ci
+        L.nvfp4_mxfp4_dequantize.argtypes = [vp, vp, i64, i64, ci, vp, vp]
+        L.nvfp4_mxfp4_gemm.restype = ci
+        L.nvfp4_mxfp4_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, vp, i64, vp]
         _lib = L
     return _lib
 
@@ -196,6 +202,22 @@ def nvfp4_quantize_2d_from_amax(w, rows, cols, ld, amax, codes_row, codes_col, s
     _check("nvfp4_quantize_2d_from_amax", lib().nvfp4_quantize_2d_from_amax(
         _p(w), rows, cols, ld, _p(amax), _p(codes_row), _p(codes_col), _p(scales), _p(scales_mma_row),
         _p(scales_mma_col), _p(global_scale), _stream(stream)))
+
+
+def nvfp4_mxfp4_quantize(x, rows, cols, ld, codes, scales, scales_mma, stream=None):
+    _check("nvfp4_mxfp4_quantize", lib().nvfp4_mxfp4_quantize(
+        _p(x), rows, cols, ld, _p(codes), _p(scales), _p(scales_mma), _stream(stream)))
+
+
+def nvfp4_mxfp4_dequantize(codes, scales, rows, cols, out_dtype, out, stream=None):
+    _check("nvfp4_mxfp4_dequantize", lib().nvfp4_mxfp4_dequantize(
+        _p(codes), _p(scales), rows, cols, out_dtype, _p(out), _stream(stream)))
+
+
+def nvfp4_mxfp4_gemm(a_codes, a_scales_mma, b_codes, b_scales_mma, M, N, K, out_dtype, c, ldc, stream=None):
+    _check("nvfp4_mxfp4_gemm", lib().nvfp4_mxfp4_gemm(
+        _p(a_codes), _p(a_scales_mma), _p(b_codes), _p(b_scales_mma), M, N, K, out_dtype, _p(c), ldc,
+        _stream(stream)))
 
 
 def nvfp4_scales_to_mma(scales, scale_mode, rows, k, scales_mma, stream=None):
@@ -314,4 +336,26 @@ def gemm(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M: int, N: in
     else:
         nvfp4_gemm(a_codes, a_scales_mma, a_gs, b_codes, b_scales_mma, b_gs, M, N, K, out_dtype, out,
                    out.stride(0), stream)
+    return out
+
+
+def mxfp4_quantize(x: torch.Tensor, plain_scales: bool = True, mma_scales: bool = True, stream=None) -> Quantized:
+    """MXFP4 quantization of a bf16 [rows x cols] tensor (32-element blocks, E8M0 scales)."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    dev = x.device
+    codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev) if plain_scales else None
+    smma = _empty_u8(nvfp4_mma_scale_bytes(rows, cols), dev) if mma_scales else None
+    nvfp4_mxfp4_quantize(x, rows, cols, x.stride(0), codes, scales, smma, stream)
+    return Quantized(codes, scales, smma, torch.ones(1, dtype=torch.float32, device=dev), rows, cols)
+
+
+def mxfp4_gemm(a: Quantized, b: Quantized, out_dtype: int = NVFP4_OUT_BF16, stream=None) -> torch.Tensor:
+    """C = A . B^T of two MXFP4 operands (K-major)."""
+    M, K, N = a.rows, a.cols, b.rows
+    dt = torch.float32 if out_dtype == NVFP4_OUT_F32 else torch.bfloat16
+    ldc = (N + 7) // 8 * 8
+    out = torch.empty(M, ldc, dtype=dt, device=a.codes.device)[:, :N]
+    nvfp4_mxfp4_gemm(a.codes, a.scales_mma, b.codes, b.scales_mma, M, N, K, out_dtype, out, out.stride(0), stream)
     return out
