@@ -107,11 +107,38 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
     return c;
 }
 
+// The ten round keys of Philox4x32-10 for one key (k0, k1): (k0 + r *
+// 0x9E3779B9, k1 + r * 0xBB67AE85), r = 0..9.  Computed once on the host and
+// passed as kernel parameters, so every round reads its key from the
+// parameter bank instead of recomputing it.
+struct PhiloxKeys {
+    uint32_t k[20];
+};
+inline PhiloxKeys philox_round_keys(uint64_t key) {
+    PhiloxKeys r;
+    uint32_t k0 = (uint32_t)key, k1 = (uint32_t)(key >> 32);
+    for (int i = 0; i < 10; ++i) {
+        r.k[2 * i] = k0;
+        r.k[2 * i + 1] = k1;
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return r;
+}
+__device__ __forceinline__ uint4 philox4x32_10_keys(uint4 c, const PhiloxKeys& keys) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+        c = make_uint4(hi1 ^ c.y ^ keys.k[2 * r], lo1, hi0 ^ c.w ^ keys.k[2 * r + 1], lo0);
+    }
+    return c;
+}
+
 // 16 random bits for the 8 output elements 8g .. 8g+7 (element e: word e/2,
-// low half for even e).
-__device__ __forceinline__ uint4 sr_bits8(uint64_t seed, uint64_t g) {
-    return philox4x32_10(make_uint4((uint32_t)g, (uint32_t)(g >> 32), 0u, 0u), (uint32_t)seed,
-                         (uint32_t)(seed >> 32));
+// low half for even e), Philox keyed by the seed whose round keys are given.
+__device__ __forceinline__ uint4 sr_bits8(const PhiloxKeys& keys, uint64_t g) {
+    return philox4x32_10_keys(make_uint4((uint32_t)g, (uint32_t)(g >> 32), 0u, 0u), keys);
 }
 // The 16 random bits u of element e: word e/2, low half for even e.
 __device__ __forceinline__ uint32_t sr_u16(const uint4& w, int e) {
@@ -141,6 +168,22 @@ __device__ __forceinline__ uint32_t rht_sign_mask(uint64_t rht_seed) {
 __device__ __forceinline__ float sr_grid(float v, uint32_t u) {
     const uint32_t t = __float_as_uint(__fmul_rz(v, 0x1p-126f)) + (u << 6);
     return __fmul_rn(__uint_as_float(t & 0xFFC00000u), 0x1p126f);
+}
+// sr_grid of two values with the two scalings done as f32x2 multiplies.
+__device__ __forceinline__ void sr_grid2(float& v0, float& v1, uint32_t u0, uint32_t u1) {
+    float s0, s1;
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 b, {%4, %4};\n\t"
+        "mul.rz.f32x2 d, a, b;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(s0), "=f"(s1)
+        : "f"(v0), "f"(v1), "f"(0x1p-126f));
+    const float r0 = __uint_as_float((__float_as_uint(s0) + (u0 << 6)) & 0xFFC00000u);
+    const float r1 = __uint_as_float((__float_as_uint(s1) + (u1 << 6)) & 0xFFC00000u);
+    const float2 q = __fmul2_rn(make_float2(r0, r1), make_float2(0x1p126f, 0x1p126f));
+    v0 = q.x;
+    v1 = q.y;
 }
 
 // Per-block scale derived from the block amax ("精度核心:两级分层缩放";

@@ -95,6 +95,7 @@ struct Params {
     const uint16_t* x;
     int64_t rows, cols, ld;
     uint64_t rht_seed, sr_seed;
+    PhiloxKeys sr_keys;           // round keys of sr_seed
     uint8_t* codes;
     uint8_t* scales;
     uint8_t* scales_mma;
@@ -162,8 +163,8 @@ __device__ __forceinline__ void rht16_regs(float y[16]) {
 // Encode one 16-block held by one thread: codes for elements 0..7 (lo) and
 // 8..15 (hi).  SR draws its bits for output elements 8g .. 8g+15.
 template <bool SR>
-__device__ __forceinline__ void encode16(const float y[16], const BlockScale& bs, uint64_t sr_seed, uint64_t g,
-                                         uint32_t& lo, uint32_t& hi) {
+__device__ __forceinline__ void encode16(const float y[16], const BlockScale& bs, const PhiloxKeys& sr_keys,
+                                         uint64_t g, uint32_t& lo, uint32_t& hi) {
     float q[16];
     if (!isinf(bs.r)) {
 #pragma unroll
@@ -177,12 +178,12 @@ __device__ __forceinline__ void encode16(const float y[16], const BlockScale& bs
         for (int i = 0; i < 16; ++i) q[i] = scaled_inf(y[i]);
     }
     if (SR) {
-        const uint4 r0 = sr_bits8(sr_seed, g);
-        const uint4 r1 = sr_bits8(sr_seed, g + 1);
+        const uint4 r0 = sr_bits8(sr_keys, g);
+        const uint4 r1 = sr_bits8(sr_keys, g + 1);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            q[i] = sr_grid(q[i], sr_u16(r0, i));
-            q[i + 8] = sr_grid(q[i + 8], sr_u16(r1, i));
+        for (int i = 0; i < 8; i += 2) {
+            sr_grid2(q[i], q[i + 1], sr_u16(r0, i), sr_u16(r0, i + 1));
+            sr_grid2(q[i + 8], q[i + 9], sr_u16(r1, i), sr_u16(r1, i + 1));
         }
     }
     lo = e2m1x8(q[0], q[1], q[2], q[3], q[4], q[5], q[6], q[7]);
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
                 // scales, which is what the padded GEMM scale layout holds.
                 const BlockScale bs = block_scale(bmax, ctx);
                 uint32_t lo, hi;
-                encode16<SR>(y, bs, p.sr_seed, (uint64_t)(rr[k] * p.cols + cc[k]) >> 3, lo, hi);
+                encode16<SR>(y, bs, p.sr_keys, (uint64_t)(rr[k] * p.cols + cc[k]) >> 3, lo, hi);
                 const int64_t b = cc[k] >> 4;
                 if (ok[k]) {
                     *reinterpret_cast<uint2*>(p.codes + rr[k] * (p.cols >> 1) + (cc[k] >> 1)) = make_uint2(lo, hi);
@@ -391,12 +392,12 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
                 const uint32_t code = c ? bs1.code : bs0.code;
                 if (SR) {
                     const uint64_t g = (uint64_t)((f0 + j) * T + t0) >> 3;
-                    const uint4 r0 = sr_bits8(p.sr_seed, g);
-                    const uint4 r1 = sr_bits8(p.sr_seed, g + 1);
+                    const uint4 r0 = sr_bits8(p.sr_keys, g);
+                    const uint4 r1 = sr_bits8(p.sr_keys, g + 1);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        q[c][i] = sr_grid(q[c][i], sr_u16(r0, i));
-                        q[c][i + 8] = sr_grid(q[c][i + 8], sr_u16(r1, i));
+                    for (int i = 0; i < 8; i += 2) {
+                        sr_grid2(q[c][i], q[c][i + 1], sr_u16(r0, i), sr_u16(r0, i + 1));
+                        sr_grid2(q[c][i + 8], q[c][i + 9], sr_u16(r1, i), sr_u16(r1, i + 1));
                     }
                 }
                 const uint32_t lo = e2m1x8(q[c][0], q[c][1], q[c][2], q[c][3], q[c][4], q[c][5], q[c][6], q[c][7]);
@@ -728,6 +729,7 @@ cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches
     p.ld = a.ld;
     p.rht_seed = a.rht_seed;
     p.sr_seed = a.sr_seed;
+    p.sr_keys = philox_round_keys(a.sr_seed);
     p.codes = a.codes;
     p.scales = a.scales;
     p.scales_mma = a.scales_mma;
