@@ -210,6 +210,21 @@ class Step:
                 events[i][1].record(stream)
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of every rank's value (replica timing: the job is as slow
+    as its slowest GPU).  One all-reduce(MAX) of a single float."""
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step_per_rank: float, world: int, ms_step: float) -> float:
+    """Whole-job throughput: every rank runs the same step on its own data
+    (weak scaling), so the job does world x the per-rank flops per step."""
+    return flops_per_step_per_rank * world / (ms_step * 1e-3) / 1e12
+
+
 def native(args):
     import torch
     import torch.distributed as dist
@@ -262,14 +277,12 @@ def native(args):
     assert N.nvfp4_get_error(s.cuda_stream) == 0
     ms_total = t0.elapsed_time(t1)
     if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+        ms_total = max_over_ranks(ms_total, dist, dev)
     ms_step = ms_total / args.steps
     per_op_ms = [statistics.mean(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(args.steps))
                  for i in range(len(ops))]
     gemm_flops = sum(o[2] for o in ops if o[1] == "gemm")
-    value = gemm_flops * world / (ms_step * 1e-3) / 1e12
+    value = job_tflops(gemm_flops, world, ms_step)
 
     hbm, bf16, bf16_sus, peak_src = peaks()
     long_region = ms_total > 2000.0

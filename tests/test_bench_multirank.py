@@ -1,0 +1,65 @@
+"""The N > 1 path of bench.py on CPU: two gloo ranks (the GPU run uses NCCL
+over the same calls).  Replicas only: the ranks exchange nothing but the
+timing, which is the maximum over ranks, and the job's throughput counts
+every rank's work; the reference arm runs on rank 0 alone."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    import datetime
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = [7.5, 9.25][rank]
+        got = bench.max_over_ranks(ms, dist, torch.device("cpu"))
+        q.put((rank, got, bench.job_tflops(23.1e12, world, got / 10)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_timing_is_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    assert [r[1] for r in res] == [9.25, 9.25]
+    # 2 ranks x 23.1 TFLOP per step in 0.925 ms per step
+    assert res[0][2] == pytest.approx(2 * 23.1e12 / 0.925e-3 / 1e12)
+
+
+def test_reference_arm_prints_on_rank0_only():
+    env = dict(os.environ, WORLD_SIZE="2", RANK="1", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0 and out.stdout.strip() == ""
+    env["RANK"], env["LOCAL_RANK"] = "0", "0"
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], env=env, capture_output=True, text=True, timeout=300)
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert out.returncode == 0 and line["impl"] == "reference" and line["n_gpus"] == 2
