@@ -194,3 +194,27 @@ def test_mlp_step_full_size():
     ah = np.concatenate([O.dequantize_f64(ga[r][0][None], ga[r][1][None], 0, sga, 1, t) for r in rows_f])
     bh = O.dequantize_f64(cb, sb, 0, sgb, h, t)
     gemm_rows_check(dw[rows_f].float().cpu().numpy(), ah, bh)
+
+
+def test_mxfp4_full_size_sampled_rows():
+    """MXFP4 of the MLP step's activation (16384 x 8192) and an MXFP4 GEMM at
+    the fprop shape: sampled rows against the oracle (MXFP4 has no tensor
+    scale, so a row's codes depend on that row alone)."""
+    T, H = G.MLP_STEP["tokens"], G.MLP_STEP["hidden"]
+    sb = G.SEED_BASE["mlp_step"]
+    x_bits = G.activation(T, H, seed=sb + 20)
+    qx = N.mxfp4_quantize(to_device_bf16(x_bits))
+    w_bits = G.weight(4096, H, seed=sb + 21)
+    qw = N.mxfp4_quantize(to_device_bf16(w_bits))
+    c = N.mxfp4_gemm(qx, qw, out_dtype=N.NVFP4_OUT_F32)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error() == 0
+    rows = sample_rows(T, seed=7)
+    codes_x, scales_x = O.mx_quantize(x_bits[rows])
+    assert np.array_equal(qx.codes.cpu().numpy()[rows], codes_x)
+    assert np.array_equal(qx.scales.cpu().numpy()[rows], scales_x)
+    cw, sw = O.mx_quantize(w_bits)
+    assert np.array_equal(qw.codes.cpu().numpy(), cw)
+    ref, s = O.mx_gemm_reference(codes_x, scales_x, cw, sw, len(rows), 4096, H)
+    err = np.abs(c.cpu().numpy()[rows].astype(np.float64) - ref)
+    assert (err <= TOL * s).all(), float((err / np.maximum(s, 1e-300)).max())
