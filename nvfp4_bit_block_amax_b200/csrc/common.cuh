@@ -128,9 +128,11 @@ inline PhiloxKeys philox_round_keys(uint64_t key) {
 __device__ __forceinline__ uint4 philox4x32_10_keys(uint4 c, const PhiloxKeys& keys) {
 #pragma unroll
     for (int r = 0; r < 10; ++r) {
-        const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
-        const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
-        c = make_uint4(hi1 ^ c.y ^ keys.k[2 * r], lo1, hi0 ^ c.w ^ keys.k[2 * r + 1], lo0);
+        // one 32 x 32 -> 64-bit multiply per word gives both halves
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c.x;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c.z;
+        c = make_uint4((uint32_t)(p1 >> 32) ^ c.y ^ keys.k[2 * r], (uint32_t)p1,
+                       (uint32_t)(p0 >> 32) ^ c.w ^ keys.k[2 * r + 1], (uint32_t)p0);
     }
     return c;
 }
