@@ -150,7 +150,7 @@ class Step:
         self.dytq = (e(f, t // 2), e(mb(f, t)))                     # wgrad A
         self.xtq = (e(h, t // 2), e(mb(h, t)))                      # wgrad B
         self.gs = torch.zeros(8, dtype=torch.float32, device=dev)
-        self.ws = torch.empty(N.nvfp4_workspace_size(0, 0), dtype=u8, device=dev)
+        self.ws = torch.empty(2 * N.nvfp4_workspace_size(0, 0), dtype=u8, device=dev)   # the dual calls need two sets
         self.y = torch.empty(t, f, dtype=bf, device=dev)
         self.dx = torch.empty(t, h, dtype=bf, device=dev)
         self.dw = torch.empty(f, h, dtype=bf, device=dev)
@@ -160,14 +160,14 @@ class Step:
         #  bytes the two-pass quantizer moves (amax pass re-reads the input), kernels launched)
         q1 = 2 + 0.5 + 1 / 16
         q2 = 2 + 0.5 + 0.5 + 2 / 16
+        # dual: one shared amax read, then one read per encode pass; two code sets written
+        qd = 2 + 2 * (0.5 + 1 / 16)
         self.ops = [
-            ("quantize_1d X (rowwise RNE)", "quant", t * h * q1, t * h * (q1 + 2), 2),
+            ("quantize_dual X (rowwise RNE + RHT X^T RNE)", "quant", t * h * qd, t * h * (qd + 4), 3),
             ("quantize_2d W (row + col codes)", "quant", f * h * q2, f * h * (q2 + 2), 2),
             ("gemm fprop", "gemm", 2.0 * t * f * h, 0, 1),
-            ("quantize_1d dY (rowwise SR)", "quant", t * f * q1, t * f * (q1 + 2), 2),
+            ("quantize_dual dY (rowwise SR + RHT dY^T SR)", "quant", t * f * qd, t * f * (qd + 4), 3),
             ("gemm dgrad", "gemm", 2.0 * t * h * f, 0, 1),
-            ("rht_quantize dY^T (SR)", "quant", t * f * q1, t * f * (q1 + 2), 2),
-            ("rht_quantize X^T (RNE)", "quant", t * h * q1, t * h * (q1 + 2), 2),
             ("gemm wgrad", "gemm", 2.0 * f * h * t, 0, 1),
         ]
 
@@ -176,7 +176,8 @@ class Step:
         t, h, f = T, H, F
         ldb = ws.numel()
         if i == 0:
-            N.nvfp4_quantize_1d(self.x, t, h, h, 0, N.NVFP4_RNE, 0, self.xq[0], None, self.xq[1], self.gp[0], ws, ldb, s)
+            N.nvfp4_quantize_dual(self.x, t, h, h, N.NVFP4_RNE, 0, self.xq[0], None, self.xq[1], self.gp[0],
+                                  self.rht_seed, 0, self.xtq[0], None, self.xtq[1], self.gp[4], ws, ldb, s)
         elif i == 1:
             N.nvfp4_quantize_2d(self.w, f, h, h, self.wq[0], self.wq[2], None, self.wq[1], self.wq[3], self.gp[1], ws,
                                 ldb, s)
@@ -184,18 +185,13 @@ class Step:
             N.nvfp4_gemm(self.xq[0], self.xq[1], self.gp[0], self.wq[0], self.wq[1], self.gp[1], t, f, h,
                          N.NVFP4_OUT_BF16, self.y, f, s)
         elif i == 3:
-            N.nvfp4_quantize_1d(self.dy, t, f, f, 0, N.NVFP4_SR, self.sr_seed, self.dyq[0], None, self.dyq[1],
-                                self.gp[2], ws, ldb, s)
+            N.nvfp4_quantize_dual(self.dy, t, f, f, N.NVFP4_SR, self.sr_seed, self.dyq[0], None, self.dyq[1],
+                                  self.gp[2], self.rht_seed, self.sr_seed + 1, self.dytq[0], None, self.dytq[1],
+                                  self.gp[3], ws, ldb, s)
         elif i == 4:
             N.nvfp4_gemm(self.dyq[0], self.dyq[1], self.gp[2], self.wq[2], self.wq[3], self.gp[1], t, h, f,
                          N.NVFP4_OUT_BF16, self.dx, h, s)
         elif i == 5:
-            N.nvfp4_rht_quantize_sr(self.dy, t, f, f, 1, self.rht_seed, N.NVFP4_SR, self.sr_seed + 1, self.dytq[0],
-                                    None, self.dytq[1], self.gp[3], ws, ldb, s)
-        elif i == 6:
-            N.nvfp4_rht_quantize_sr(self.x, t, h, h, 1, self.rht_seed, N.NVFP4_RNE, 0, self.xtq[0], None,
-                                    self.xtq[1], self.gp[4], ws, ldb, s)
-        elif i == 7:
             N.nvfp4_gemm(self.dytq[0], self.dytq[1], self.gp[3], self.xtq[0], self.xtq[1], self.gp[4], f, h, t,
                          N.NVFP4_OUT_BF16, self.dw, h, s)
 

@@ -165,6 +165,25 @@ nvfp4_status nvfp4_rht_quantize_sr(const void* x, int64_t rows, int64_t cols, in
                                    uint8_t* scales, uint8_t* scales_mma, float* global_scale,
                                    void* workspace, size_t ws_bytes, void* stream);
 
+/* Both GEMM roles of one tensor in one call ["Empat pengaman" -- the
+ * gradient and the activation are each needed row-wise (fprop/dgrad) and,
+ * rotated, column-wise (wgrad); "NVFP4 Is a Scaling System", "Where speed and
+ * accuracy claims can fail" -- quantization work counts]:
+ *   Q1 = x, 1D along cols (as nvfp4_quantize_1d with transpose = 0, sr_seed),
+ *   Q2 = RHT(x^T), 1D along rows (as nvfp4_rht_quantize_sr with transpose = 1,
+ *        rht_seed, sr_seed_t),
+ *   both with `rounding`.  Outputs are bit-identical to the two separate
+ *   calls.  The two amax passes share one read of x (the rotated and the
+ *   plain maxima are reduced together), so x is read three times instead of
+ *   four.  rows and cols multiples of 16; workspace >= 2 *
+ *   nvfp4_workspace_size(rows, cols) bytes; codes [rows x cols/2], codes_t
+ *   [cols x rows/2], scales / scales_mma as the single calls. */
+nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ld, int rounding,
+                                 uint64_t sr_seed, uint8_t* codes, uint8_t* scales, uint8_t* scales_mma,
+                                 float* global_scale, uint64_t rht_seed, uint64_t sr_seed_t, uint8_t* codes_t,
+                                 uint8_t* scales_t, uint8_t* scales_mma_t, float* global_scale_t, void* workspace,
+                                 size_t ws_bytes, void* stream);
+
 /* 2D (16x16 tile) quantization of a weight, RNE ["2D block scaling for
  * weights" (How does MVFP4 make 4-bit AI training work?); "Empat pengaman" --
  * one scale per 16x16 block makes rowwise and columnwise quantization

@@ -184,6 +184,46 @@ static nvfp4_status quantize_2d_impl(const void* w, int64_t rows, int64_t cols, 
     return from_cuda(e);
 }
 
+nvfp4_status nvfp4_quantize_dual(const void* x, int64_t rows, int64_t cols, int64_t ld, int rounding,
+                                 uint64_t sr_seed, uint8_t* codes, uint8_t* scales, uint8_t* scales_mma,
+                                 float* global_scale, uint64_t rht_seed, uint64_t sr_seed_t, uint8_t* codes_t,
+                                 uint8_t* scales_t, uint8_t* scales_mma_t, float* global_scale_t, void* workspace,
+                                 size_t ws_bytes, void* stream) {
+    // both halves must pass the single-call checks; the workspace holds two sets of partials
+    nvfp4_status st = check_quant_common(x, rows, cols, ld, 0, rounding, codes, scales, scales_mma, global_scale,
+                                         workspace, ws_bytes);
+    if (st != NVFP4_OK) return st;
+    st = check_quant_common(x, rows, cols, ld, 1, rounding, codes_t, scales_t, scales_mma_t, global_scale_t,
+                            workspace, ws_bytes);
+    if (st != NVFP4_OK) return st;
+    if (ws_bytes < 2 * kWorkspaceBytes) return NVFP4_ERR_WORKSPACE;
+    QuantArgs r{}, t{};
+    r.x = t.x = static_cast<const uint16_t*>(x);
+    r.rows = t.rows = rows;
+    r.cols = t.cols = cols;
+    r.ld = t.ld = ld;
+    r.rounding = t.rounding = rounding;
+    r.sr_seed = sr_seed;
+    r.codes = codes;
+    r.scales = scales;
+    r.scales_mma = scales_mma;
+    r.global_scale = global_scale;
+    r.partials = static_cast<uint32_t*>(workspace) + kMaxPartials;
+    t.transpose = 1;
+    t.rht = 1;
+    t.rht_seed = rht_seed;
+    t.sr_seed = sr_seed_t;
+    t.codes = codes_t;
+    t.scales = scales_t;
+    t.scales_mma = scales_mma_t;
+    t.global_scale = global_scale_t;
+    t.partials = static_cast<uint32_t*>(workspace);
+    int n = 0;
+    cudaError_t e = launch_quantize_dual(r, t, static_cast<cudaStream_t>(stream), &n);
+    g_launches += n;
+    return from_cuda(e);
+}
+
 nvfp4_status nvfp4_quantize_2d(const void* w, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes_row,
                                uint8_t* codes_col, uint8_t* scales, uint8_t* scales_mma_row,
                                uint8_t* scales_mma_col, float* global_scale, void* workspace, size_t ws_bytes,

@@ -42,6 +42,7 @@ struct Quant2dArgs {
 
 cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches);
 cudaError_t launch_quantize_2d(const Quant2dArgs& a, cudaStream_t s, int* launches);
+cudaError_t launch_quantize_dual(const QuantArgs& r, const QuantArgs& t, cudaStream_t s, int* launches);
 cudaError_t launch_quantize_1d_noalloc(const QuantArgs& a, cudaStream_t s, int* launches, bool* too_big);
 int noalloc_capacity();
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, int scale_mode, const float* gs,

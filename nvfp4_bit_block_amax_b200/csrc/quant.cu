@@ -103,6 +103,7 @@ struct Params {
     float* global_scale;
     uint32_t* partials;
     int n_partials;
+    uint32_t* partials2;          // amax pass of the dual quantizer: plain |x| maxima here too
 };
 
 // Global scale from the amax partials; block 0 publishes it.
@@ -325,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
     const int64_t ntt = (T + 127) >> 7, nft = (F + 255) >> 8;
     const int64_t ntiles = ntt * nft;
     const int64_t kb = T >> 4;
-    uint32_t amax_bits = 0;
+    uint32_t amax_bits = 0, plain_acc = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int64_t tt = tile / nft, ft = tile - tt * nft;
         const int64_t t0 = tt * 128 + warp * 16;
@@ -335,6 +336,11 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             v[i] = ok ? ldg_stream(p.x + (t0 + i) * p.ld + f0) : make_uint4(0u, 0u, 0u, 0u);
+        if (AMAX_ONLY && p.partials2) {   // the un-rotated amax from the same read
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                plain_acc = absmax2(absmax2(absmax2(absmax2(plain_acc, v[i].x), v[i].y), v[i].z), v[i].w);
+        }
 #pragma unroll
         for (int jp = 0; jp < 4; ++jp) {
             float2 y[16];
@@ -432,7 +438,13 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
         }
         __syncthreads();
     }
-    if (AMAX_ONLY) write_partial(amax_bits, p.partials);
+    if (AMAX_ONLY) {
+        write_partial(amax_bits, p.partials);
+        if (p.partials2) {
+            __syncthreads();   // write_partial's shared scratch is reused
+            write_partial(absmax2_fold(plain_acc), p.partials2);
+        }
+    }
 }
 
 // ------------------------------------------------------------ 2D (16x16) ---
@@ -750,6 +762,65 @@ cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches
     }
     if (a.rht) return sr ? run_cols<true, true>(p, g, s, launches) : run_cols<true, false>(p, g, s, launches);
     return sr ? run_cols<false, true>(p, g, s, launches) : run_cols<false, false>(p, g, s, launches);
+}
+
+// Both GEMM roles of one tensor from one amax read: Q = x (1D along the
+// rows, args r) and Q = RHT(x^T) (args t).  The transposed amax pass also
+// reduces the plain |x| maxima (second half of the workspace), which the
+// row-wise encode pass then folds; the transposed encode pass folds the
+// rotated ones.  Three launches instead of four, one full read saved.
+cudaError_t launch_quantize_dual(const QuantArgs& r, const QuantArgs& t, cudaStream_t s, int* launches) {
+    Params pt{};
+    pt.x = t.x;
+    pt.rows = t.rows;
+    pt.cols = t.cols;
+    pt.ld = t.ld;
+    pt.rht_seed = t.rht_seed;
+    pt.sr_seed = t.sr_seed;
+    pt.sr_keys = philox_round_keys(t.sr_seed);
+    pt.codes = t.codes;
+    pt.scales = t.scales;
+    pt.scales_mma = t.scales_mma;
+    pt.chunks_k = mma_chunks_k(t.rows);
+    pt.global_scale = t.global_scale;
+    pt.partials = t.partials;
+    pt.partials2 = r.partials;
+    Params pr{};
+    pr.x = r.x;
+    pr.rows = r.rows;
+    pr.cols = r.cols;
+    pr.ld = r.ld;
+    pr.sr_seed = r.sr_seed;
+    pr.sr_keys = philox_round_keys(r.sr_seed);
+    pr.codes = r.codes;
+    pr.scales = r.scales;
+    pr.scales_mma = r.scales_mma;
+    pr.chunks_k = mma_chunks_k(r.cols);
+    pr.global_scale = r.global_scale;
+    pr.partials = r.partials;
+    if (r.scales_mma && ((r.rows % 128) || ((r.cols / 16) % 4))) {
+        cudaError_t e = cudaMemsetAsync(r.scales_mma, 0, mma_scale_bytes(r.rows, r.cols), s);
+        if (e != cudaSuccess) return e;
+    }
+    if (t.scales_mma && ((t.cols % 128) || ((t.rows / 16) % 4))) {
+        cudaError_t e = cudaMemsetAsync(t.scales_mma, 0, mma_scale_bytes(t.cols, t.rows), s);
+        if (e != cudaSuccess) return e;
+    }
+    const bool sr_r = r.rounding == 1, sr_t = t.rounding == 1;
+    const int64_t tiles = ((t.rows + 127) >> 7) * ((t.cols + 255) >> 8);
+    const int gc = sr_t ? grid_for(cols_kernel<true, true, false>, tiles) : grid_for(cols_kernel<true, false, false>, tiles);
+    cols_kernel<true, false, true><<<gc, kThreads, 0, s>>>(pt);
+    pt.n_partials = gc;
+    pr.n_partials = gc;
+    pt.partials2 = nullptr;
+    const int64_t units = r.rows * ((r.cols + 511) >> 9);
+    const int64_t wneed = (units + 1) / 2;
+    if (sr_r) rows_kernel<false, true, false><<<grid_for(rows_kernel<false, true, false>, (wneed + 7) / 8), kThreads, 0, s>>>(pr);
+    else rows_kernel<false, false, false><<<grid_for(rows_kernel<false, false, false>, (wneed + 7) / 8), kThreads, 0, s>>>(pr);
+    if (sr_t) cols_kernel<true, true, false><<<gc, kThreads, 0, s>>>(pt);
+    else cols_kernel<true, false, false><<<gc, kThreads, 0, s>>>(pt);
+    *launches += 3;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_2d(const Quant2dArgs& a, cudaStream_t s, int* launches) {

@@ -34,6 +34,7 @@ EXPORTS = (
     "nvfp4_scales_to_mma", "nvfp4_kernel_launches", "nvfp4_get_error", "nvfp4_quantize_1d_noalloc",
     "nvfp4_selftest_wait_timeout", "nvfp4_quantize_1d_from_amax", "nvfp4_quantize_2d_from_amax",
     "nvfp4_gemm_amax", "nvfp4_mxfp4_quantize", "nvfp4_mxfp4_dequantize", "nvfp4_mxfp4_gemm",
+    "nvfp4_quantize_dual",
 )
 
 _lib = None
@@ -92,6 +93,9 @@ def lib():
         L.nvfp4_mxfp4_quantize.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp]
         L.nvfp4_mxfp4_dequantize.restype = ci
         L.nvfp4_mxfp4_dequantize.argtypes = [vp, vp, i64, i64, ci, vp, vp]
+        L.nvfp4_quantize_dual.restype = ci
+        L.nvfp4_quantize_dual.argtypes = [vp, i64, i64, i64, ci, u64, vp, vp, vp, vp, u64, u64, vp, vp, vp, vp, vp,
+                                          sz, vp]
         L.nvfp4_mxfp4_gemm.restype = ci
         L.nvfp4_mxfp4_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, ci, vp, i64, vp]
         _lib = L
@@ -162,6 +166,14 @@ def nvfp4_rht_quantize_sr(x, rows, cols, ld, transpose, rht_seed, rounding, sr_s
     _check("nvfp4_rht_quantize_sr", lib().nvfp4_rht_quantize_sr(
         _p(x), rows, cols, ld, transpose, rht_seed, rounding, sr_seed, _p(codes), _p(scales), _p(scales_mma),
         _p(global_scale), _p(workspace), ws_bytes, _stream(stream)))
+
+
+def nvfp4_quantize_dual(x, rows, cols, ld, rounding, sr_seed, codes, scales, scales_mma, global_scale, rht_seed,
+                        sr_seed_t, codes_t, scales_t, scales_mma_t, global_scale_t, workspace, ws_bytes, stream=None):
+    _check("nvfp4_quantize_dual", lib().nvfp4_quantize_dual(
+        _p(x), rows, cols, ld, rounding, sr_seed, _p(codes), _p(scales), _p(scales_mma), _p(global_scale), rht_seed,
+        sr_seed_t, _p(codes_t), _p(scales_t), _p(scales_mma_t), _p(global_scale_t), _p(workspace), ws_bytes,
+        _stream(stream)))
 
 
 def nvfp4_quantize_2d(w, rows, cols, ld, codes_row, codes_col, scales, scales_mma_row, scales_mma_col,
@@ -359,3 +371,24 @@ def mxfp4_gemm(a: Quantized, b: Quantized, out_dtype: int = NVFP4_OUT_BF16, stre
     out = torch.empty(M, ldc, dtype=dt, device=a.codes.device)[:, :N]
     nvfp4_mxfp4_gemm(a.codes, a.scales_mma, b.codes, b.scales_mma, M, N, K, out_dtype, out, out.stride(0), stream)
     return out
+
+
+def quantize_dual(x: torch.Tensor, rounding: int = NVFP4_RNE, sr_seed: int = 0, rht_seed: int = 0,
+                  sr_seed_t: int = 0, stream=None):
+    """(Q1, Q2): x row-wise and RHT(x^T), from one shared amax read."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    dev = x.device
+    q1 = Quantized(torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev),
+                   torch.empty(rows, cols // 16, dtype=torch.uint8, device=dev),
+                   _empty_u8(nvfp4_mma_scale_bytes(rows, cols), dev), torch.empty(1, dtype=torch.float32, device=dev),
+                   rows, cols)
+    q2 = Quantized(torch.empty(cols, rows // 2, dtype=torch.uint8, device=dev),
+                   torch.empty(cols, rows // 16, dtype=torch.uint8, device=dev),
+                   _empty_u8(nvfp4_mma_scale_bytes(cols, rows), dev), torch.empty(1, dtype=torch.float32, device=dev),
+                   cols, rows)
+    ws = torch.empty(2 * nvfp4_workspace_size(rows, cols), dtype=torch.uint8, device=dev)
+    nvfp4_quantize_dual(x, rows, cols, x.stride(0), rounding, sr_seed, q1.codes, q1.scales, q1.scales_mma,
+                        q1.global_scale, rht_seed, sr_seed_t, q2.codes, q2.scales, q2.scales_mma, q2.global_scale,
+                        ws, ws.numel(), stream)
+    return q1, q2

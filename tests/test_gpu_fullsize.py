@@ -218,3 +218,24 @@ def test_mxfp4_full_size_sampled_rows():
     ref, s = O.mx_gemm_reference(codes_x, scales_x, cw, sw, len(rows), 4096, H)
     err = np.abs(c.cpu().numpy()[rows].astype(np.float64) - ref)
     assert (err <= TOL * s).all(), float((err / np.maximum(s, 1e-300)).max())
+
+
+def test_mlp_step_dual_quantizer_full_size():
+    """The step's dual quantizer calls at full size (X RNE, dY SR) are
+    bit-identical to the separate calls that the step test checks against the
+    oracle."""
+    t, h, f = G.MLP_STEP["tokens"], G.MLP_STEP["hidden"], G.MLP_STEP["ffn"]
+    seed, rs, ss = G.seeds("mlp_step")
+    for bits, rnd, s1, s2 in ((G.activation(t, h, seed), N.NVFP4_RNE, 0, 0),
+                              (G.gradient(t, f, seed + 2), N.NVFP4_SR, ss, ss + 1)):
+        xd = to_device_bf16(bits)
+        q1, q2 = N.quantize_dual(xd, rounding=rnd, sr_seed=s1, rht_seed=rs, sr_seed_t=s2)
+        a = N.quantize_1d(xd, rounding=rnd, sr_seed=s1)
+        b = N.quantize_1d(xd, transpose=True, rht=True, rht_seed=rs, rounding=rnd, sr_seed=s2)
+        torch.cuda.synchronize()
+        assert N.nvfp4_get_error() == 0
+        for u, v in ((q1.codes, a.codes), (q1.scales_mma, a.scales_mma), (q1.global_scale, a.global_scale),
+                     (q2.codes, b.codes), (q2.scales_mma, b.scales_mma), (q2.global_scale, b.global_scale)):
+            assert torch.equal(u, v)
+        del xd, q1, q2, a, b
+        torch.cuda.empty_cache()
