@@ -53,7 +53,7 @@ def parse():
     ap.add_argument("--op", default=None,
                     choices=["gemm", "gemm_amax", "quantize_1d", "quantize_1d_sr", "quantize_2d", "rht_t_sr",
                              "rht_t_rne", "quantize_1d_from_amax", "quantize_2d_from_amax", "mx_quantize",
-                             "mx_gemm",
+                             "mx_gemm", "quantize_dual", "quantize_dual_sr",
                              "dequantize"],
                     help="time one kernel family alone on --shape (profiling mode)")
     ap.add_argument("--shape", default=None, help="M,N,K for gemm; rows,cols otherwise")
@@ -538,6 +538,15 @@ def micro(args):
             sm2 = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)
             fn = lambda: N.nvfp4_quantize_2d_from_amax(x, R, C, C, amax, codes, cc, None, smma, sm2, gs, s)
             work = R * C * (2 + 0.5 + 0.5 + 2 / 16)
+        elif args.op in ("quantize_dual", "quantize_dual_sr"):
+            rnd = N.NVFP4_SR if args.op.endswith("sr") else N.NVFP4_RNE
+            ct = torch.empty(C, R // 2, dtype=torch.uint8, device=dev)
+            smt = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)
+            gt = torch.empty(1, dtype=torch.float32, device=dev)
+            ws2 = torch.empty(2 * N.nvfp4_workspace_size(R, C), dtype=torch.uint8, device=dev)
+            fn = lambda: N.nvfp4_quantize_dual(x, R, C, C, rnd, 7, codes, None, smma, gs, 5, 8, ct, None, smt, gt,
+                                               ws2, ws2.numel(), s)
+            work = R * C * (2 + 2 * (0.5 + 1 / 16))
         elif args.op == "mx_quantize":
             fn = lambda: N.nvfp4_mxfp4_quantize(x, R, C, C, codes, None, smma, s)
             work = R * C * (2 + 0.5 + 1 / 32)
