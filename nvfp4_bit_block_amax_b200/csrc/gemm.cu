@@ -437,6 +437,9 @@ __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int ha
     return true;
 }
 
+// MX: MXFP4 operands (scale_vec::2X, UE8M0); a compile-time choice, so the
+// MMA issue loop carries no branch for it.
+template <bool MX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, KParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -527,7 +530,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
             int s = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            const uint32_t idesc = kIdesc | (p.mx ? kIdescUe8m0 : 0u);
+            const uint32_t idesc = kIdesc | (MX ? kIdescUe8m0 : 0u);
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 if (!mbar_wait(bar_tempty, acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
@@ -543,7 +546,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
                     const uint32_t sfb_col = sfa_col + 16;
                     for (int j = 0; j < nk; ++j)
                         tc_mma_nvf4(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32), idesc,
-                                    sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0, p.mx);
+                                    sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0, MX);
                     tc_commit(bar_empty + 8 * s);
                     if (++s == STAGES) { s = 0; phase ^= 1; }
                 }
@@ -775,6 +778,7 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
     return true;
 }
 
+template <bool MX>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, KParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -865,7 +869,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
             int s = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            const uint32_t idesc = kIdescPair | (p.mx ? kIdescUe8m0 : 0u);
+            const uint32_t idesc = kIdescPair | (MX ? kIdescUe8m0 : 0u);
             for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
                 if (!mbar_wait_cluster(bar_tempty, acc_phase ^ 1, abort_flag)) break;
                 tc_fence_after();
@@ -881,7 +885,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                     const uint32_t sfb_col = sfa_col + 16;
                     for (int j = 0; j < nk; ++j)
                         tc_mma_nvf4_pair(tmem + ACC_COL, desc_sw128(a_addr + j * 32), desc_sw128(b_addr + j * 32),
-                                         idesc, sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0, p.mx);
+                                         idesc, sfa_col + 4 * j, sfb_col + 8 * j, (kb | j) != 0, MX);
                     tc_commit_pair(bar_empty + 8 * s);
                     if (++s == P_STAGES) { s = 0; phase ^= 1; }
                 }
@@ -1058,9 +1062,12 @@ DeviceInfo device_info() {
     if (!d.sms) {
         int n = 0;
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cudaFuncSetAttribute(gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-        cudaFuncSetAttribute(gemm_nvf4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
-        cudaFuncSetAttribute(gemm_nvf4_pair_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+        for (auto k : {gemm_nvf4_kernel<false>, gemm_nvf4_kernel<true>})
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        for (auto k : {gemm_nvf4_pair_kernel<false>, gemm_nvf4_pair_kernel<true>}) {
+            cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_BYTES);
+            cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (n / 2));
         cfg.blockDim = dim3(NUM_THREADS);
@@ -1073,7 +1080,8 @@ DeviceInfo device_info() {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int clusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_nvf4_pair_kernel, &cfg) != cudaSuccess || clusters < 1) {
+        if (cudaOccupancyMaxActiveClusters(&clusters, gemm_nvf4_pair_kernel<false>, &cfg) != cudaSuccess ||
+            clusters < 1) {
             cudaGetLastError();
             clusters = n / 2;
         }
@@ -1123,7 +1131,8 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
         p.group_m = group_for(BM, g.K, p.tiles_m);
         const int tiles = p.tiles_m * p.tiles_n;
         const int grid = tiles < dev.sms ? tiles : dev.sms;
-        gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+        if (p.mx) gemm_nvf4_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+        else gemm_nvf4_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, p);
         return cudaGetLastError();
     }
     // CTA pairs: 256 x 256 tiles, each CTA loads 128-row boxes of A and B
@@ -1146,7 +1155,8 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel, ma, mb, p);
+    return p.mx ? cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<true>, ma, mb, p)
+                : cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<false>, ma, mb, p);
 }
 
 unsigned int read_and_clear_error_word(cudaStream_t s, cudaError_t* err) {
