@@ -329,7 +329,7 @@ def native(args):
         "kernels": kernels,
         "roofline": {"bound": "tensor", "achieved": round(gemm_ach, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(gemm_ach / fp4_peak, 4), "traffic": traffic,
-                     "kernel": "gemm_nvf4_kernel (3 GEMMs, mean over launches)",
+                     "kernel": "gemm_nvf4_pair_kernel (3 GEMMs, mean over launches)",
                      "peak_source": f"{peak_src} {'sustained' if long_region else 'burst'} bf16 x {FP4_OVER_BF16} "
                                     "(nominal FP4/BF16 dense ratio)"},
         "clocks": clk,
