@@ -260,12 +260,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return d;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-    return v;
-}
-
 // Reduce the per-CTA amax partials (binary32 bits of non-negative maxima) to
 // the tensor amax; every thread of the block gets it.
 __device__ __forceinline__ float reduce_partials(const uint32_t* __restrict__ partials, int n) {

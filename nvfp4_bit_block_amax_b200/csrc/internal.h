@@ -8,7 +8,6 @@ namespace nvfp4 {
 
 // Grid of the amax pass: one partial maximum per CTA, reduced by every CTA of
 // the quantize pass that follows on the same stream.
-int amax_grid(int64_t units);
 constexpr int kMaxPartials = 4096;
 
 struct QuantArgs {

@@ -731,8 +731,6 @@ cudaError_t run_cols(Params p, const float* given, cudaStream_t s, int* launches
 
 }  // namespace
 
-int amax_grid(int64_t units) { return (int)std::min<int64_t>(units, kMaxPartials); }
-
 cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches) {
     Params p{};
     p.x = a.x;
