@@ -39,6 +39,10 @@
  *  - The RHT is 16 points, y = (1/4) * H16 * (d . x), H16 the Sylvester
  *    matrix in natural order, applied per 16-chunk along the quantized axis,
  *    d a +-1 vector drawn from Philox; amax is taken of the rotated values.
+ *    Larger orders n = 32, 64, 128 (the Sylvester recursion goes on to any
+ *    power of two): the same butterflies for h = 1 .. n/2, then one multiply
+ *    by RN(1/sqrt(n)); the 16-element quantization blocks stay as they are,
+ *    n/16 of them per chunk.
  *  - Stochastic rounding uses 16 random bits per element from Philox keyed by
  *    (seed, element index in the quantized output layout).
  *  NOTE: nothing here calls, links or includes the CUDA library.
@@ -177,35 +181,51 @@ uint32_t nvfp4o_sr_bits(uint64_t seed, uint64_t i) {
 }
 
 /* RHT sign vector [P2 "随机 Hadamard 变换" -- a random diagonal of signs]:
- * word 0 of Philox at counter (0, 0, 1, 0), key from rht_seed; d_j = -1 iff
- * bit j is set.  Writes 16 entries of +-1. */
-void nvfp4o_rht_signs(uint64_t rht_seed, float d[16]) {
+ * Philox at counter (0, 0, 1, 0), key from rht_seed; d_j = -1 iff bit
+ * (j mod 32) of output word floor(j / 32) is set.  Writes n entries of +-1,
+ * n <= 128 (one Philox call gives 128 bits); the first 16 entries do not
+ * depend on n. */
+void nvfp4o_rht_signs_n(uint64_t rht_seed, int n, float* d) {
     uint32_t ctr[4] = {0u, 0u, 1u, 0u};
     uint32_t key[2] = {(uint32_t)rht_seed, (uint32_t)(rht_seed >> 32)};
     uint32_t out[4];
     nvfp4o_philox4x32_10(ctr, key, out);
-    for (int j = 0; j < 16; ++j) d[j] = ((out[0] >> j) & 1u) ? -1.0f : 1.0f;
+    for (int j = 0; j < n; ++j) d[j] = ((out[j / 32] >> (j % 32)) & 1u) ? -1.0f : 1.0f;
 }
 
-/* 16-point random Hadamard transform of one chunk [P2 "构造 Hadamard 矩阵的方法"
- * (Sylvester recursion: four H_n blocks, lower-right negated) and "为什么不用
- * Conference 矩阵" (fast transform by butterflies, additions and subtractions
- * only)]: y = d . x; for h = 1, 2, 4, 8 replace each pair (y_i, y_{i+h}) with
- * i & h == 0 by (y_i + y_{i+h}, y_i - y_{i+h}); then multiply by 1/4 so that
- * the transform (1/4) H16 D is orthogonal. */
-void nvfp4o_rht16(const float x[16], const float d[16], float y[16]) {
-    float t[16];
-    for (int j = 0; j < 16; ++j) t[j] = d[j] * x[j];
-    for (int h = 1; h < 16; h <<= 1) {
-        for (int i = 0; i < 16; ++i) {
+/* The 16-point sign vector (word 0, bits 0..15). */
+void nvfp4o_rht_signs(uint64_t rht_seed, float d[16]) { nvfp4o_rht_signs_n(rht_seed, 16, d); }
+
+/* Normalisation of the n-point transform: 1/sqrt(n) rounded to binary32
+ * (a power of two for n = 16, 64; RN(sqrt(2)) * 2^-3 and * 2^-4 for n = 32
+ * and 128), so that RN(1/sqrt(n)) * H_n * D is orthogonal up to one
+ * rounding of the factor. */
+float nvfp4o_rht_norm(int n) { return (float)(1.0 / sqrt((double)n)); }
+
+/* n-point random Hadamard transform of one chunk, n a power of two in
+ * [16, 128] [P2 "构造 Hadamard 矩阵的方法" (Sylvester recursion: four H_n
+ * blocks, lower-right negated, so H_n[i][j] = (-1)^popcount(i & j)) and
+ * "为什么不用 Conference 矩阵" (fast transform by butterflies, additions and
+ * subtractions only)]: y = d . x; for h = 1, 2, 4, ..., n/2 replace each pair
+ * (y_i, y_{i+h}) with i & h == 0 by (y_i + y_{i+h}, y_i - y_{i+h}); then
+ * multiply every entry by nvfp4o_rht_norm(n). */
+void nvfp4o_rht_n(const float* x, const float* d, int n, float* y) {
+    float t[128];
+    for (int j = 0; j < n; ++j) t[j] = d[j] * x[j];
+    for (int h = 1; h < n; h <<= 1) {
+        for (int i = 0; i < n; ++i) {
             if (i & h) continue;
             float a = t[i], b = t[i + h];
             t[i] = a + b;
             t[i + h] = a - b;
         }
     }
-    for (int j = 0; j < 16; ++j) y[j] = t[j] * 0.25f;
+    float c = nvfp4o_rht_norm(n);
+    for (int j = 0; j < n; ++j) y[j] = t[j] * c;
 }
+
+/* The 16-point transform, y = (1/4) H16 (d . x). */
+void nvfp4o_rht16(const float x[16], const float d[16], float y[16]) { nvfp4o_rht_n(x, d, 16, y); }
 
 /* ------------------------------------------------------------------------ */
 /* Global (tensor) scale [P3 "Anatomi NVFP4"]: amax / (448 * 6). */
@@ -240,29 +260,33 @@ static float q_at(const uint16_t* x, int64_t ld, int transpose, int64_t r, int64
     return transpose ? bf16_to_float(x[c * ld + r]) : bf16_to_float(x[r * ld + c]);
 }
 
-/* Row r of Q after the optional RHT, 16 values per chunk. */
-static void q_chunk(const uint16_t* x, int64_t ld, int transpose, int rht, const float d[16],
-                    int64_t r, int64_t c0, float y[16]) {
-    float t[16];
-    for (int j = 0; j < 16; ++j) t[j] = q_at(x, ld, transpose, r, c0 + j);
-    if (rht) nvfp4o_rht16(t, d, y);
-    else memcpy(y, t, sizeof t);
+/* Row r of Q, columns c0 .. c0+n-1, after the n-point RHT when rht_n != 0
+ * (n = rht_n, c0 a multiple of it); without RHT, n = 16. */
+static void q_chunk(const uint16_t* x, int64_t ld, int transpose, int rht_n, const float* d,
+                    int64_t r, int64_t c0, float* y) {
+    int n = rht_n ? rht_n : 16;
+    float t[128];
+    for (int j = 0; j < n; ++j) t[j] = q_at(x, ld, transpose, r, c0 + j);
+    if (rht_n) nvfp4o_rht_n(t, d, rht_n, y);
+    else memcpy(y, t, sizeof(float) * (size_t)n);
 }
 
 /* Tensor amax [P3 "Anatomi NVFP4"; P5 "Why two levels" -- the global scale
  * comes from the tensor's maximum absolute value before the block maxima],
- * over Q (rotated when rht != 0). */
-float nvfp4o_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
-                  int rht, uint64_t rht_seed) {
+ * over Q (rotated by the rht_n-point transform when rht_n != 0; the length of
+ * a Q row must then be a multiple of rht_n). */
+float nvfp4o_amax_n(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                    int rht_n, uint64_t rht_seed) {
     int64_t qr = transpose ? cols : rows, qc = transpose ? rows : cols;
-    float d[16];
+    int n = rht_n ? rht_n : 16;
+    float d[128];
     float a = 0.0f;
-    if (rht) nvfp4o_rht_signs(rht_seed, d);
+    if (rht_n) nvfp4o_rht_signs_n(rht_seed, rht_n, d);
     for (int64_t r = 0; r < qr; ++r) {
-        for (int64_t c0 = 0; c0 + 16 <= qc; c0 += 16) {
-            float y[16];
-            q_chunk(x, ld, transpose, rht, d, r, c0, y);
-            for (int j = 0; j < 16; ++j) {
+        for (int64_t c0 = 0; c0 + n <= qc; c0 += n) {
+            float y[128];
+            q_chunk(x, ld, transpose, rht_n, d, r, c0, y);
+            for (int j = 0; j < n; ++j) {
                 float m = fabsf(y[j]);
                 if (m > a) a = m;
             }
@@ -271,52 +295,79 @@ float nvfp4o_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int
     return a;
 }
 
+float nvfp4o_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                  int rht, uint64_t rht_seed) {
+    return nvfp4o_amax_n(x, rows, cols, ld, transpose, rht ? 16 : 0, rht_seed);
+}
+
 /* 1D quantization (16 consecutive elements of a Q row share one E4M3 scale)
  * of Q rows [r_begin, r_end), given the tensor's global scale.  codes points
  * at the codes of row r_begin ([r_end - r_begin] x Q_cols/2), scales at its
  * scales ([r_end - r_begin] x Q_cols/16).  rounding 0 = RNE (weights and
- * activations), 1 = SR (gradients) [P2 "随机舍入:为什么只用在梯度上"]. */
-void nvfp4o_quantize_1d_rows(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
-                             int transpose, int rht, uint64_t rht_seed, int rounding,
-                             uint64_t sr_seed, float s_global, int64_t r_begin, int64_t r_end,
-                             uint8_t* codes, uint8_t* scales) {
+ * activations), 1 = SR (gradients) [P2 "随机舍入:为什么只用在梯度上"].
+ * rht_n != 0: Q rows are first rotated chunk by chunk (rht_n points, a
+ * multiple of 16); each chunk then holds rht_n/16 blocks. */
+void nvfp4o_quantize_1d_rows_n(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                               int transpose, int rht_n, uint64_t rht_seed, int rounding,
+                               uint64_t sr_seed, float s_global, int64_t r_begin, int64_t r_end,
+                               uint8_t* codes, uint8_t* scales) {
     int64_t qc = transpose ? rows : cols;
-    float d[16];
-    if (rht) nvfp4o_rht_signs(rht_seed, d);
+    int n = rht_n ? rht_n : 16;
+    float d[128];
+    if (rht_n) nvfp4o_rht_signs_n(rht_seed, rht_n, d);
     for (int64_t r = r_begin; r < r_end; ++r) {
-        for (int64_t c0 = 0; c0 + 16 <= qc; c0 += 16) {
-            float y[16];
-            q_chunk(x, ld, transpose, rht, d, r, c0, y);
-            float b = 0.0f;
-            for (int j = 0; j < 16; ++j) {
-                float m = fabsf(y[j]);
-                if (m > b) b = m;
-            }
-            int sc = nvfp4o_block_scale_code(b, s_global);
-            float s_dec = (float)nvfp4o_e4m3_value(sc);
-            scales[(r - r_begin) * (qc / 16) + c0 / 16] = (uint8_t)sc;
-            for (int j = 0; j < 16; ++j) {
-                uint64_t idx = (uint64_t)(r * qc + c0 + j);
-                uint32_t u = rounding ? nvfp4o_sr_bits(sr_seed, idx) : 0u;
-                int code = nvfp4o_encode_element(y[j], s_dec, s_global, rounding, u);
-                uint8_t* byte = &codes[(r - r_begin) * (qc / 2) + (c0 + j) / 2];
-                if (((c0 + j) & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | code);
-                else *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
+        for (int64_t c0 = 0; c0 + n <= qc; c0 += n) {
+            float ychunk[128];
+            q_chunk(x, ld, transpose, rht_n, d, r, c0, ychunk);
+            for (int b0 = 0; b0 < n; b0 += 16) {
+                const float* y = ychunk + b0;
+                int64_t cb = c0 + b0;
+                float b = 0.0f;
+                for (int j = 0; j < 16; ++j) {
+                    float m = fabsf(y[j]);
+                    if (m > b) b = m;
+                }
+                int sc = nvfp4o_block_scale_code(b, s_global);
+                float s_dec = (float)nvfp4o_e4m3_value(sc);
+                scales[(r - r_begin) * (qc / 16) + cb / 16] = (uint8_t)sc;
+                for (int j = 0; j < 16; ++j) {
+                    uint64_t idx = (uint64_t)(r * qc + cb + j);
+                    uint32_t u = rounding ? nvfp4o_sr_bits(sr_seed, idx) : 0u;
+                    int code = nvfp4o_encode_element(y[j], s_dec, s_global, rounding, u);
+                    uint8_t* byte = &codes[(r - r_begin) * (qc / 2) + (cb + j) / 2];
+                    if (((cb + j) & 1) == 0) *byte = (uint8_t)((*byte & 0xF0) | code);
+                    else *byte = (uint8_t)((*byte & 0x0F) | (code << 4));
+                }
             }
         }
     }
 }
 
+void nvfp4o_quantize_1d_rows(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                             int transpose, int rht, uint64_t rht_seed, int rounding,
+                             uint64_t sr_seed, float s_global, int64_t r_begin, int64_t r_end,
+                             uint8_t* codes, uint8_t* scales) {
+    nvfp4o_quantize_1d_rows_n(x, rows, cols, ld, transpose, rht ? 16 : 0, rht_seed, rounding, sr_seed,
+                              s_global, r_begin, r_end, codes, scales);
+}
+
 /* Whole-tensor 1D quantization: amax, global scale, then every row. */
+void nvfp4o_quantize_1d_n(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                          int rht_n, uint64_t rht_seed, int rounding, uint64_t sr_seed,
+                          uint8_t* codes, uint8_t* scales, float* global_scale) {
+    float a = nvfp4o_amax_n(x, rows, cols, ld, transpose, rht_n, rht_seed);
+    float sg = nvfp4o_global_scale(a);
+    int64_t qr = transpose ? cols : rows;
+    nvfp4o_quantize_1d_rows_n(x, rows, cols, ld, transpose, rht_n, rht_seed, rounding, sr_seed, sg, 0, qr,
+                              codes, scales);
+    *global_scale = sg;
+}
+
 void nvfp4o_quantize_1d(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
                         int rht, uint64_t rht_seed, int rounding, uint64_t sr_seed,
                         uint8_t* codes, uint8_t* scales, float* global_scale) {
-    float a = nvfp4o_amax(x, rows, cols, ld, transpose, rht, rht_seed);
-    float sg = nvfp4o_global_scale(a);
-    int64_t qr = transpose ? cols : rows;
-    nvfp4o_quantize_1d_rows(x, rows, cols, ld, transpose, rht, rht_seed, rounding, sr_seed, sg, 0, qr,
-                            codes, scales);
-    *global_scale = sg;
+    nvfp4o_quantize_1d_n(x, rows, cols, ld, transpose, rht ? 16 : 0, rht_seed, rounding, sr_seed, codes, scales,
+                         global_scale);
 }
 
 /* 2D quantization of a weight [P1 "2D block scaling for weights"; P3 "Empat

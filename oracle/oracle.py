@@ -62,6 +62,18 @@ def lib():
             L.nvfp4o_rht_signs.argtypes = [u64, vp]
             L.nvfp4o_rht16.restype = None
             L.nvfp4o_rht16.argtypes = [vp, vp, vp]
+            L.nvfp4o_rht_signs_n.restype = None
+            L.nvfp4o_rht_signs_n.argtypes = [u64, ci, vp]
+            L.nvfp4o_rht_norm.restype = fp
+            L.nvfp4o_rht_norm.argtypes = [ci]
+            L.nvfp4o_rht_n.restype = None
+            L.nvfp4o_rht_n.argtypes = [vp, vp, ci, vp]
+            L.nvfp4o_amax_n.restype = fp
+            L.nvfp4o_amax_n.argtypes = [vp, i64, i64, i64, ci, ci, u64]
+            L.nvfp4o_quantize_1d_rows_n.restype = None
+            L.nvfp4o_quantize_1d_rows_n.argtypes = [vp, i64, i64, i64, ci, ci, u64, ci, u64, fp, i64, i64, vp, vp]
+            L.nvfp4o_quantize_1d_n.restype = None
+            L.nvfp4o_quantize_1d_n.argtypes = [vp, i64, i64, i64, ci, ci, u64, ci, u64, vp, vp, vp]
             L.nvfp4o_global_scale.restype = fp
             L.nvfp4o_global_scale.argtypes = [fp]
             L.nvfp4o_block_scale_code.restype = ci
@@ -197,36 +209,78 @@ def rht16(x, d) -> np.ndarray:
     return y
 
 
+RHT_ORDERS = (16, 32, 64, 128)
+
+
+def rht_signs_n(rht_seed: int, n: int) -> np.ndarray:
+    """The n-point sign vector (n <= 128): d_j = -1 iff bit j % 32 of Philox word j // 32."""
+    if n not in RHT_ORDERS:
+        raise ValueError("RHT order must be one of 16, 32, 64, 128")
+    d = np.zeros(n, dtype=np.float32)
+    lib().nvfp4o_rht_signs_n(int(rht_seed), int(n), _ptr(d))
+    return d
+
+
+def rht_norm(n: int) -> np.float32:
+    """RN(1/sqrt(n)) in binary32, the factor applied after the butterflies."""
+    return np.float32(lib().nvfp4o_rht_norm(int(n)))
+
+
+def rht_n(x, d) -> np.ndarray:
+    """One n-point chunk of the random Hadamard transform, RN(1/sqrt(n)) H_n (d . x), n = len(x)."""
+    xx = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    dd = np.ascontiguousarray(np.asarray(d, dtype=np.float32))
+    n = xx.size
+    if n not in RHT_ORDERS or dd.size != n:
+        raise ValueError("RHT order must be one of 16, 32, 64, 128")
+    y = np.zeros(n, dtype=np.float32)
+    lib().nvfp4o_rht_n(_ptr(xx), _ptr(dd), int(n), _ptr(y))
+    return y
+
+
+def _rht_n_arg(rht: bool, rht_order: int) -> int:
+    if not rht:
+        return 0
+    if rht_order not in RHT_ORDERS:
+        raise ValueError("RHT order must be one of 16, 32, 64, 128")
+    return int(rht_order)
+
+
 # ---------------------------------------------------------------- tensors --
-def amax(x: np.ndarray, transpose: bool = False, rht: bool = False, rht_seed: int = 0) -> float:
+def amax(x: np.ndarray, transpose: bool = False, rht: bool = False, rht_seed: int = 0,
+         rht_order: int = 16) -> float:
     """Tensor amax of the quantized tensor Q (x or x^T, rotated when rht)."""
     x = _bf16(x)
     rows, cols = x.shape
-    return lib().nvfp4o_amax(_ptr(x), rows, cols, x.strides[0] // 2, int(transpose), int(rht), int(rht_seed))
+    return lib().nvfp4o_amax_n(_ptr(x), rows, cols, x.strides[0] // 2, int(transpose),
+                               _rht_n_arg(rht, rht_order), int(rht_seed))
 
 
 def quantize_1d(x: np.ndarray, transpose: bool = False, rht: bool = False, rht_seed: int = 0,
-                rounding: int = 0, sr_seed: int = 0):
+                rounding: int = 0, sr_seed: int = 0, rht_order: int = 16):
     """Whole-tensor 1D NVFP4 quantization of bf16 x [rows x cols].
 
     Returns (codes [Qr x Qc/2] uint8, scales [Qr x Qc/16] uint8, s_global float32),
-    Q = x^T when ``transpose``.  Rounding 0 = RNE, 1 = SR.
+    Q = x^T when ``transpose``.  Rounding 0 = RNE, 1 = SR.  With ``rht`` the
+    Q rows are rotated in chunks of ``rht_order`` points (Qc a multiple of it).
     """
     x = np.ascontiguousarray(_bf16(x))
     rows, cols = x.shape
     qr, qc = (cols, rows) if transpose else (rows, cols)
-    if qc % 16:
-        raise ValueError("quantized rows must hold a multiple of 16 elements")
+    n = _rht_n_arg(rht, rht_order)
+    if qc % 16 or (n and qc % n):
+        raise ValueError("quantized rows must hold a multiple of 16 (and of the RHT order) elements")
     codes = np.zeros((qr, qc // 2), dtype=np.uint8)
     scales = np.zeros((qr, qc // 16), dtype=np.uint8)
     sg = np.zeros(1, dtype=np.float32)
-    lib().nvfp4o_quantize_1d(_ptr(x), rows, cols, cols, int(transpose), int(rht), int(rht_seed),
-                             int(rounding), int(sr_seed), _ptr(codes), _ptr(scales), _ptr(sg))
+    lib().nvfp4o_quantize_1d_n(_ptr(x), rows, cols, cols, int(transpose), n, int(rht_seed),
+                               int(rounding), int(sr_seed), _ptr(codes), _ptr(scales), _ptr(sg))
     return codes, scales, np.float32(sg[0])
 
 
 def quantize_1d_rows(x: np.ndarray, s_global: float, row_ids, transpose: bool = False,
-                     rht: bool = False, rht_seed: int = 0, rounding: int = 0, sr_seed: int = 0):
+                     rht: bool = False, rht_seed: int = 0, rounding: int = 0, sr_seed: int = 0,
+                     rht_order: int = 16):
     """1D quantization of selected rows of Q given the tensor's global scale.
 
     Returns dicts {row: (codes_row, scales_row)} for each row id (sampling of
@@ -236,14 +290,17 @@ def quantize_1d_rows(x: np.ndarray, s_global: float, row_ids, transpose: bool = 
         raise ValueError("contiguous input expected")
     rows, cols = x.shape
     qr, qc = (cols, rows) if transpose else (rows, cols)
+    n = _rht_n_arg(rht, rht_order)
+    if n and qc % n:
+        raise ValueError("quantized rows must hold a multiple of the RHT order")
     out = {}
     codes = np.zeros((1, qc // 2), dtype=np.uint8)
     scales = np.zeros((1, qc // 16), dtype=np.uint8)
     for r in row_ids:
         r = int(r)
-        lib().nvfp4o_quantize_1d_rows(_ptr(x), rows, cols, cols, int(transpose), int(rht), int(rht_seed),
-                                      int(rounding), int(sr_seed), float(s_global), r, r + 1,
-                                      _ptr(codes), _ptr(scales))
+        lib().nvfp4o_quantize_1d_rows_n(_ptr(x), rows, cols, cols, int(transpose), n, int(rht_seed),
+                                        int(rounding), int(sr_seed), float(s_global), r, r + 1,
+                                        _ptr(codes), _ptr(scales))
         out[r] = (codes[0].copy(), scales[0].copy())
     return out
 
