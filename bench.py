@@ -54,9 +54,11 @@ def parse():
                     choices=["gemm", "gemm_amax", "quantize_1d", "quantize_1d_sr", "quantize_2d", "rht_t_sr",
                              "rht_t_rne", "quantize_1d_from_amax", "quantize_2d_from_amax", "mx_quantize",
                              "mx_gemm", "quantize_dual", "quantize_dual_sr",
-                             "dequantize"],
+                             "dequantize", "rht_sr", "rht_rne"],
                     help="time one kernel family alone on --shape (profiling mode)")
     ap.add_argument("--shape", default=None, help="M,N,K for gemm; rows,cols otherwise")
+    ap.add_argument("--rht-order", type=int, default=16, choices=[16, 32, 64, 128],
+                    help="points of the Hadamard transform for the rht_* ops (rht_t_*: transposed)")
     return ap.parse_args()
 
 
@@ -607,7 +609,9 @@ def micro(args):
             work = R * C * (0.5 + 1 / 16 + 2)
         else:
             rnd = N.NVFP4_SR if args.op.endswith("sr") else N.NVFP4_RNE
-            fn = lambda: N.nvfp4_rht_quantize_sr(x, R, C, C, 1, 5, rnd, 6, codes, None, smma, gs, ws, ws.numel(), s)
+            n = args.rht_order
+            fn = lambda: N.nvfp4_rht_quantize_n(x, R, C, C, int(tr), n, 5, rnd, 6, codes, None, smma, gs, ws,
+                                                ws.numel(), s)
             work = R * C * (2 + 0.5 + 1 / 16)
     for _ in range(args.warmup):
         fn()
@@ -621,7 +625,8 @@ def micro(args):
     assert N.nvfp4_get_error(s.cuda_stream) == 0
     ms = e0.elapsed_time(e1) / args.steps
     scale = 1e12 if unit == "TFLOP/s" else 1e9
-    print(json.dumps({"op": args.op, "shape": dims, "ms": round(ms, 4), "throughput": round(work / (ms * 1e-3) / scale, 1),
+    print(json.dumps({"op": args.op, "shape": dims, **({"rht_order": args.rht_order} if args.op.startswith("rht")
+                                                         else {}), "ms": round(ms, 4), "throughput": round(work / (ms * 1e-3) / scale, 1),
                       "unit": unit, "note": "profiling mode (one op alone), not a bench line"}), flush=True)
 
 

@@ -165,6 +165,27 @@ nvfp4_status nvfp4_rht_quantize_sr(const void* x, int64_t rows, int64_t cols, in
                                    uint8_t* scales, uint8_t* scales_mma, float* global_scale,
                                    void* workspace, size_t ws_bytes, void* stream);
 
+/* The same with an RHT of larger order ["MXFP4 和 NVFP4 的区别", "构造
+ * Hadamard 矩阵的方法" -- the Sylvester recursion gives H for every power of
+ * two; "为什么不用 Conference 矩阵,而用 Hadamard" -- the fast transform is
+ * butterflies of additions and subtractions].
+ *   rht_order      n = 16, 32, 64 or 128 (16 is nvfp4_rht_quantize_sr).
+ *                  Every n-chunk of a Q row is replaced by
+ *                  y = c_n H_n (d . chunk): butterflies h = 1, 2, ..., n/2 as
+ *                  above, then one binary32 multiply by c_n = RN(1/sqrt(n))
+ *                  (1/4, RN(sqrt 2)/8, 1/8, RN(sqrt 2)/16); d_j = -1 iff bit
+ *                  j % 32 of word j / 32 of the same Philox output (the
+ *                  16-point signs are its first 16).  Blocks stay 16
+ *                  elements, n/16 per chunk.
+ *   The length of a Q row (cols, or rows when transpose = 1) must be a
+ *   multiple of n: NVFP4_ERR_UNSUPPORTED_SHAPE otherwise; another order is
+ *   NVFP4_ERR_INVALID_ARG.  Other arguments, layouts and errors as
+ *   nvfp4_rht_quantize_sr. */
+nvfp4_status nvfp4_rht_quantize_n(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                                  int rht_order, uint64_t rht_seed, int rounding, uint64_t sr_seed,
+                                  uint8_t* codes, uint8_t* scales, uint8_t* scales_mma, float* global_scale,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
 /* Both GEMM roles of one tensor in one call ["Empat pengaman" -- the
  * gradient and the activation are each needed row-wise (fprop/dgrad) and,
  * rotated, column-wise (wgrad); "NVFP4 Is a Scaling System", "Where speed and

@@ -71,10 +71,15 @@ long long nvfp4_kernel_launches(void) { return g_launches.load(); }
 static nvfp4_status quantize_1d_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose, int rht,
                                      uint64_t rht_seed, int rounding, uint64_t sr_seed, uint8_t* codes,
                                      uint8_t* scales, uint8_t* scales_mma, float* global_scale, void* workspace,
-                                     size_t ws_bytes, void* stream, const float* given_amax = nullptr) {
+                                     size_t ws_bytes, void* stream, const float* given_amax = nullptr,
+                                     int rht_order = 16) {
     nvfp4_status st = check_quant_common(x, rows, cols, ld, transpose, rounding, codes, scales, scales_mma,
                                          global_scale, workspace, ws_bytes);
     if (st != NVFP4_OK) return st;
+    if (rht) {
+        if (rht_order != 16 && rht_order != 32 && rht_order != 64 && rht_order != 128) return NVFP4_ERR_INVALID_ARG;
+        if ((transpose ? rows : cols) % rht_order) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    }
     QuantArgs a{};
     a.x = static_cast<const uint16_t*>(x);
     a.rows = rows;
@@ -82,6 +87,7 @@ static nvfp4_status quantize_1d_impl(const void* x, int64_t rows, int64_t cols, 
     a.ld = ld;
     a.transpose = transpose;
     a.rht = rht;
+    a.rht_order = rht_order;
     a.rht_seed = rht_seed;
     a.rounding = rounding;
     a.sr_seed = sr_seed;
@@ -150,6 +156,14 @@ nvfp4_status nvfp4_rht_quantize_sr(const void* x, int64_t rows, int64_t cols, in
                                    size_t ws_bytes, void* stream) {
     return quantize_1d_impl(x, rows, cols, ld, transpose, 1, rht_seed, rounding, sr_seed, codes, scales,
                             scales_mma, global_scale, workspace, ws_bytes, stream);
+}
+
+nvfp4_status nvfp4_rht_quantize_n(const void* x, int64_t rows, int64_t cols, int64_t ld, int transpose,
+                                  int rht_order, uint64_t rht_seed, int rounding, uint64_t sr_seed, uint8_t* codes,
+                                  uint8_t* scales, uint8_t* scales_mma, float* global_scale, void* workspace,
+                                  size_t ws_bytes, void* stream) {
+    return quantize_1d_impl(x, rows, cols, ld, transpose, 1, rht_seed, rounding, sr_seed, codes, scales,
+                            scales_mma, global_scale, workspace, ws_bytes, stream, nullptr, rht_order);
 }
 
 static nvfp4_status quantize_2d_impl(const void* w, int64_t rows, int64_t cols, int64_t ld, uint8_t* codes_row,

@@ -154,6 +154,24 @@ __device__ __forceinline__ uint32_t rht_sign_mask(uint64_t rht_seed) {
     return philox4x32_10(make_uint4(0u, 0u, 1u, 0u), (uint32_t)rht_seed, (uint32_t)(rht_seed >> 32)).x & 0xFFFFu;
 }
 
+// Signs of an n-point RHT, n <= 128 ("构造 Hadamard 矩阵的方法": the Sylvester
+// recursion continues to any power of two): d_j = -1 <=> bit j % 32 of word
+// j / 32 of the same Philox output, so the 16-point signs are its first 16.
+// Returns the 16-bit mask of positions base .. base+15 (base a multiple of 16).
+__device__ __forceinline__ uint32_t rht_sign_mask_at(uint64_t rht_seed, int base) {
+    const uint4 w = philox4x32_10(make_uint4(0u, 0u, 1u, 0u), (uint32_t)rht_seed, (uint32_t)(rht_seed >> 32));
+    const int k = base >> 5;
+    const uint32_t word = k == 0 ? w.x : k == 1 ? w.y : k == 2 ? w.z : w.w;
+    return (word >> (base & 31)) & 0xFFFFu;
+}
+
+// Normalisation of the (16 << LOGM)-point transform: RN(1/sqrt(n)) in binary32
+// (1/4, RN(sqrt 2)/8, 1/8, RN(sqrt 2)/16), applied once after the butterflies.
+template <int LOGM>
+__device__ __forceinline__ constexpr float rht_norm() {
+    return LOGM == 0 ? 0.25f : LOGM == 1 ? 0x1.6a09e6p-3f : LOGM == 2 ? 0.125f : 0x1.6a09e6p-4f;
+}
+
 // Stochastic rounding onto the E2M1 grid of one scaled value v (finite):
 // between neighbours lo <= |v| < hi, f = floor(p * 2^16) with
 // p = (|v| - lo) / (hi - lo), round up iff f + u >= 2^16; results above 6

@@ -14,7 +14,8 @@ struct QuantArgs {
     const uint16_t* x;
     int64_t rows, cols, ld;       // input [rows x cols], row stride ld (elements)
     int transpose;                // Q = x (0) or x^T (1)
-    int rht;                      // 16-point RHT along Q rows
+    int rht;                      // RHT along Q rows
+    int rht_order;                // its order: 16 (0 also means 16), 32, 64 or 128
     uint64_t rht_seed;
     int rounding;                 // 0 RNE, 1 SR
     uint64_t sr_seed;

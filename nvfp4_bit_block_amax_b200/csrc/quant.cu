@@ -129,10 +129,10 @@ __device__ __forceinline__ void load_block(const uint16_t* p, bool a32, uint32_t
     }
 }
 
-// 16-point RHT of one chunk held by one thread: signs (exact), butterflies
-// h = 1, 2, 4, 8 (pairs of independent butterflies packed into f32x2 adds),
-// then the factor 1/4.
-__device__ __forceinline__ void rht16_regs(float y[16]) {
+// Butterflies h = 1, 2, 4, 8 of a 16-point RHT chunk held by one thread
+// (pairs of independent butterflies packed into f32x2 adds); the signs are
+// applied by the caller.
+__device__ __forceinline__ void rht16_butterflies(float y[16]) {
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1) {
         int idx[8];
@@ -153,11 +153,36 @@ __device__ __forceinline__ void rht16_regs(float y[16]) {
             y[i1 + h] = dif.y;
         }
     }
+}
+
+__device__ __forceinline__ void scale_regs(float y[16], float c) {
 #pragma unroll
     for (int i = 0; i < 16; i += 2) {
-        const float2 v = __fmul2_rn(make_float2(y[i], y[i + 1]), make_float2(0.25f, 0.25f));
+        const float2 v = __fmul2_rn(make_float2(y[i], y[i + 1]), make_float2(c, c));
         y[i] = v.x;
         y[i + 1] = v.y;
+    }
+}
+
+// The butterflies h = 16, 32, .. of a (16 << LOGM)-point RHT whose 16-point
+// pieces sit in 2^LOGM consecutive lanes (piece index = lane bits 0..LOGM-1):
+// the lane with bit s clear keeps a + b, its partner a - b, a being the
+// lower piece's value -- the order and rounding of the sequential butterflies.
+template <int LOGM>
+__device__ __forceinline__ void rht_cross_lanes(float y[16], int lane) {
+#pragma unroll
+    for (int s = 0; s < LOGM; ++s) {
+        // upper: o + (-y) = a - b; lower: o + y = a + b (addition commutes,
+        // the sign flip is exact)
+        const float sg = ((lane >> s) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            const float2 o = make_float2(__shfl_xor_sync(0xFFFFFFFFu, y[i], 1 << s),
+                                         __shfl_xor_sync(0xFFFFFFFFu, y[i + 1], 1 << s));
+            const float2 v = __fadd2_rn(o, __fmul2_rn(make_float2(y[i], y[i + 1]), make_float2(sg, sg)));
+            y[i] = v.x;
+            y[i + 1] = v.y;
+        }
     }
 }
 
@@ -194,7 +219,9 @@ __device__ __forceinline__ void encode16(const float y[16], const BlockScale& bs
 // ------------------------------------------------- rowwise 1D (Q = x) --------
 // One thread per 16-block: a warp takes 512 consecutive columns of a Q row
 // (32 blocks) per unit, consecutive units per warp, 2 units in flight.
-template <bool RHT, bool SR, bool AMAX_ONLY>
+// RHT of order 16 << LOGM: a chunk is 2^LOGM consecutive lanes (Q rows hold
+// a multiple of the order, so a chunk never straddles the end of a row).
+template <bool RHT, bool SR, bool AMAX_ONLY, int LOGM = 0>
 __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
     __shared__ float s_rtab[128];
     ScaleCtx ctx{};
@@ -203,14 +230,15 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
         global_scales(p, sg, t);
         ctx = make_scale_ctx(sg, t, s_rtab);
     }
+    const int lane = threadIdx.x & 31;
     uint32_t sw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (RHT) {
-        const uint32_t d = rht_sign_mask(p.rht_seed);
+        const uint32_t d = LOGM == 0 ? rht_sign_mask(p.rht_seed)
+                                     : rht_sign_mask_at(p.rht_seed, 16 * (lane & ((1 << LOGM) - 1)));
 #pragma unroll
         for (int k = 0; k < 8; ++k)
             sw[k] = (((d >> (2 * k)) & 1u) ? 0x8000u : 0u) | (((d >> (2 * k + 1)) & 1u) ? 0x80000000u : 0u);
     }
-    const int lane = threadIdx.x & 31;
     const int64_t upr = (p.cols + 511) >> 9;
     const int64_t total = p.rows * upr;
     const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
@@ -256,7 +284,9 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
                         y[2 * j] = bf16_lo(ww);
                         y[2 * j + 1] = bf16_hi(ww);
                     }
-                    rht16_regs(y);
+                    rht16_butterflies(y);
+                    if (LOGM > 0) rht_cross_lanes<LOGM>(y, lane);
+                    scale_regs(y, rht_norm<LOGM>());
                     bmax = 0.0f;
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) bmax = max3f(bmax, fabsf(y[j]), fabsf(y[j + 1]));
@@ -309,7 +339,11 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
 // lane: 8 features, so a thread holds 8 whole blocks (one per feature) and
 // the RHT runs in registers.  Codes are staged in shared memory and written
 // as 8-byte row segments of Q.
-template <bool RHT, bool SR, bool AMAX_ONLY>
+// RHT of order 16 << LOGM (LOGM <= 3): the same tile, mapped so that the
+// pieces of a chunk share a warp -- warp w: features 32w .. 32w+31; lane:
+// 16-token piece lane >> 2, 8 features from 8 * (lane & 3) -- and the
+// butterflies h >= 16 are shuffles between lanes lane ^ 4, ^ 8, ^ 16.
+template <bool RHT, bool SR, bool AMAX_ONLY, int LOGM = 0>
 __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
     __shared__ __align__(16) uint8_t s_codes[AMAX_ONLY ? 16 : 256 * 64];
     __shared__ __align__(16) uint8_t s_sc[AMAX_ONLY ? 1 : 256][8];   // [feature in tile][token block in tile]
@@ -320,8 +354,12 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
         global_scales(p, sg, t);
         ctx = make_scale_ctx(sg, t, s_rtab);
     }
-    const uint32_t dmask = RHT ? rht_sign_mask(p.rht_seed) : 0u;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int piece = LOGM == 0 ? warp : (lane >> 2);                     // 16-token block in the tile
+    const int fl0 = LOGM == 0 ? lane * 8 : warp * 32 + (lane & 3) * 8;    // first of 8 features in the tile
+    const uint32_t dmask = !RHT ? 0u
+                           : LOGM == 0 ? rht_sign_mask(p.rht_seed)
+                                       : rht_sign_mask_at(p.rht_seed, 16 * (piece & ((1 << LOGM) - 1)));
     const int64_t T = p.rows, F = p.cols;
     const int64_t ntt = (T + 127) >> 7, nft = (F + 255) >> 8;
     const int64_t ntiles = ntt * nft;
@@ -329,8 +367,8 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
     uint32_t amax_bits = 0, plain_acc = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
         const int64_t tt = tile / nft, ft = tile - tt * nft;
-        const int64_t t0 = tt * 128 + warp * 16;
-        const int64_t f0 = ft * 256 + lane * 8;
+        const int64_t t0 = tt * 128 + piece * 16;
+        const int64_t f0 = ft * 256 + fl0;
         const bool ok = (t0 < T) && (f0 < F);
         uint4 v[16];
 #pragma unroll
@@ -362,7 +400,20 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
                     }
                 }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) y[i] = __fmul2_rn(y[i], make_float2(0.25f, 0.25f));
+                for (int s = 0; s < LOGM; ++s) {
+                    // lower piece: o + y = a + b; upper: o + (-y) = a - b
+                    // (addition commutes, the sign flip is exact)
+                    const float sg = ((piece >> s) & 1) ? -1.0f : 1.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 o = make_float2(__shfl_xor_sync(0xFFFFFFFFu, y[i].x, 4 << s),
+                                                     __shfl_xor_sync(0xFFFFFFFFu, y[i].y, 4 << s));
+                        y[i] = __fadd2_rn(o, __fmul2_rn(y[i], make_float2(sg, sg)));
+                    }
+                }
+                constexpr float c = rht_norm<LOGM>();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) y[i] = __fmul2_rn(y[i], make_float2(c, c));
             }
             float bm0 = 0.0f, bm1 = 0.0f;
 #pragma unroll
@@ -409,9 +460,10 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
                 const uint32_t lo = e2m1x8(q[c][0], q[c][1], q[c][2], q[c][3], q[c][4], q[c][5], q[c][6], q[c][7]);
                 const uint32_t hi =
                     e2m1x8(q[c][8], q[c][9], q[c][10], q[c][11], q[c][12], q[c][13], q[c][14], q[c][15]);
-                const int srow = lane * 8 + j;
-                *reinterpret_cast<uint2*>(s_codes + srow * 64 + ((warp ^ (lane & 7)) * 8)) = make_uint2(lo, hi);
-                s_sc[srow][warp] = ok ? (uint8_t)code : (uint8_t)0;
+                const int srow = fl0 + j;
+                const int key = LOGM == 0 ? (lane & 7) : ((srow >> 3) & 7);   // = (srow >> 3) & 7
+                *reinterpret_cast<uint2*>(s_codes + srow * 64 + ((piece ^ key) * 8)) = make_uint2(lo, hi);
+                s_sc[srow][piece] = ok ? (uint8_t)code : (uint8_t)0;
                 if (ok && p.scales) p.scales[(f0 + j) * kb + (t0 >> 4)] = (uint8_t)code;
             }
         }
@@ -690,43 +742,53 @@ int launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
     return g;
 }
 
-template <bool RHT, bool SR>
+template <bool RHT, bool SR, int LOGM = 0>
 cudaError_t run_rows(Params p, const float* given, cudaStream_t s, int* launches) {
     const int64_t units = p.rows * ((p.cols + 511) >> 9);
     const int64_t warps_needed = (units + 1) / 2;
-    const int g = grid_for(rows_kernel<RHT, SR, false>, (warps_needed + 7) / 8);
+    const int g = grid_for(rows_kernel<RHT, SR, false, LOGM>, (warps_needed + 7) / 8);
     if (given) {   // the tensor amax is known: it is the single partial
         p.partials = const_cast<uint32_t*>(reinterpret_cast<const uint32_t*>(given));
         p.n_partials = 1;
         *launches -= 1;
     } else if (RHT) {
         p.n_partials = g;
-        rows_kernel<true, false, true><<<g, kThreads, 0, s>>>(p);
+        rows_kernel<true, false, true, LOGM><<<g, kThreads, 0, s>>>(p);
     } else {
         p.n_partials = launch_amax_plain(p.x, p.rows, p.cols, p.ld, p.partials, s);
     }
-    rows_kernel<RHT, SR, false><<<g, kThreads, 0, s>>>(p);
+    rows_kernel<RHT, SR, false, LOGM><<<g, kThreads, 0, s>>>(p);
     *launches += 2;
     return cudaGetLastError();
 }
 
-template <bool RHT, bool SR>
+template <bool RHT, bool SR, int LOGM = 0>
 cudaError_t run_cols(Params p, const float* given, cudaStream_t s, int* launches) {
     const int64_t tiles = ((p.rows + 127) >> 7) * ((p.cols + 255) >> 8);
-    const int g = grid_for(cols_kernel<RHT, SR, false>, tiles);
+    const int g = grid_for(cols_kernel<RHT, SR, false, LOGM>, tiles);
     if (given) {
         p.partials = const_cast<uint32_t*>(reinterpret_cast<const uint32_t*>(given));
         p.n_partials = 1;
         *launches -= 1;
     } else if (RHT) {
         p.n_partials = g;
-        cols_kernel<true, false, true><<<g, kThreads, 0, s>>>(p);
+        cols_kernel<true, false, true, LOGM><<<g, kThreads, 0, s>>>(p);
     } else {
         p.n_partials = launch_amax_plain(p.x, p.rows, p.cols, p.ld, p.partials, s);
     }
-    cols_kernel<RHT, SR, false><<<g, kThreads, 0, s>>>(p);
+    cols_kernel<RHT, SR, false, LOGM><<<g, kThreads, 0, s>>>(p);
     *launches += 2;
     return cudaGetLastError();
+}
+
+// RHT quantizers by order: log2(order / 16) as a template argument.
+template <int LOGM>
+cudaError_t run_rht(const QuantArgs& a, const Params& p, cudaStream_t s, int* launches) {
+    const bool sr = a.rounding == 1;
+    const float* g = a.given_amax;
+    if (!a.transpose)
+        return sr ? run_rows<true, true, LOGM>(p, g, s, launches) : run_rows<true, false, LOGM>(p, g, s, launches);
+    return sr ? run_cols<true, true, LOGM>(p, g, s, launches) : run_cols<true, false, LOGM>(p, g, s, launches);
 }
 
 }  // namespace
@@ -754,11 +816,16 @@ cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches
     }
     const bool sr = a.rounding == 1;
     const float* g = a.given_amax;
-    if (!a.transpose) {
-        if (a.rht) return sr ? run_rows<true, true>(p, g, s, launches) : run_rows<true, false>(p, g, s, launches);
-        return sr ? run_rows<false, true>(p, g, s, launches) : run_rows<false, false>(p, g, s, launches);
+    if (a.rht) {
+        switch (a.rht_order) {
+            case 32: return run_rht<1>(a, p, s, launches);
+            case 64: return run_rht<2>(a, p, s, launches);
+            case 128: return run_rht<3>(a, p, s, launches);
+            default: return run_rht<0>(a, p, s, launches);
+        }
     }
-    if (a.rht) return sr ? run_cols<true, true>(p, g, s, launches) : run_cols<true, false>(p, g, s, launches);
+    if (!a.transpose)
+        return sr ? run_rows<false, true>(p, g, s, launches) : run_rows<false, false>(p, g, s, launches);
     return sr ? run_cols<false, true>(p, g, s, launches) : run_cols<false, false>(p, g, s, launches);
 }
 

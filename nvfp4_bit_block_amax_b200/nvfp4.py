@@ -34,7 +34,7 @@ EXPORTS = (
     "nvfp4_scales_to_mma", "nvfp4_kernel_launches", "nvfp4_get_error", "nvfp4_quantize_1d_noalloc",
     "nvfp4_selftest_wait_timeout", "nvfp4_quantize_1d_from_amax", "nvfp4_quantize_2d_from_amax",
     "nvfp4_gemm_amax", "nvfp4_mxfp4_quantize", "nvfp4_mxfp4_dequantize", "nvfp4_mxfp4_gemm",
-    "nvfp4_quantize_dual",
+    "nvfp4_quantize_dual", "nvfp4_rht_quantize_n",
 )
 
 _lib = None
@@ -69,6 +69,8 @@ def lib():
         L.nvfp4_quantize_1d_noalloc.argtypes = [vp, i64, i64, i64, ci, ci, u64, vp, vp, vp, vp, vp]
         L.nvfp4_rht_quantize_sr.restype = ci
         L.nvfp4_rht_quantize_sr.argtypes = [vp, i64, i64, i64, ci, u64, ci, u64, vp, vp, vp, vp, vp, sz, vp]
+        L.nvfp4_rht_quantize_n.restype = ci
+        L.nvfp4_rht_quantize_n.argtypes = [vp, i64, i64, i64, ci, ci, u64, ci, u64, vp, vp, vp, vp, vp, sz, vp]
         L.nvfp4_quantize_2d.restype = ci
         L.nvfp4_quantize_2d.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.nvfp4_dequantize.restype = ci
@@ -166,6 +168,13 @@ def nvfp4_rht_quantize_sr(x, rows, cols, ld, transpose, rht_seed, rounding, sr_s
     _check("nvfp4_rht_quantize_sr", lib().nvfp4_rht_quantize_sr(
         _p(x), rows, cols, ld, transpose, rht_seed, rounding, sr_seed, _p(codes), _p(scales), _p(scales_mma),
         _p(global_scale), _p(workspace), ws_bytes, _stream(stream)))
+
+
+def nvfp4_rht_quantize_n(x, rows, cols, ld, transpose, rht_order, rht_seed, rounding, sr_seed, codes, scales,
+                         scales_mma, global_scale, workspace, ws_bytes, stream=None):
+    _check("nvfp4_rht_quantize_n", lib().nvfp4_rht_quantize_n(
+        _p(x), rows, cols, ld, transpose, rht_order, rht_seed, rounding, sr_seed, _p(codes), _p(scales),
+        _p(scales_mma), _p(global_scale), _p(workspace), ws_bytes, _stream(stream)))
 
 
 def nvfp4_quantize_dual(x, rows, cols, ld, rounding, sr_seed, codes, scales, scales_mma, global_scale, rht_seed,
@@ -280,9 +289,10 @@ def _empty_u8(n, device):
 
 def quantize_1d(x: torch.Tensor, transpose: bool = False, rounding: int = NVFP4_RNE, sr_seed: int = 0,
                 rht: bool = False, rht_seed: int = 0, plain_scales: bool = True, mma_scales: bool = True,
-                stream=None, amax: Optional[torch.Tensor] = None) -> Quantized:
+                stream=None, amax: Optional[torch.Tensor] = None, rht_order: int = 16) -> Quantized:
     """Quantize a bf16 [rows x cols] tensor (or its transpose) with 16-element blocks.
-    With `amax` (a device float holding max |x|) the amax pass is skipped."""
+    With `amax` (a device float holding max |x|) the amax pass is skipped;
+    with `rht` the Q rows are rotated in chunks of `rht_order` points."""
     assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
     rows, cols = x.shape
     qr, qc = (cols, rows) if transpose else (rows, cols)
@@ -296,6 +306,9 @@ def quantize_1d(x: torch.Tensor, transpose: bool = False, rounding: int = NVFP4_
         assert not rht, "the amax of the rotated tensor is not known to a producer"
         nvfp4_quantize_1d_from_amax(x, rows, cols, x.stride(0), int(transpose), rounding, sr_seed, amax, codes,
                                     scales, smma, gs, stream)
+    elif rht and rht_order != 16:
+        nvfp4_rht_quantize_n(x, rows, cols, x.stride(0), int(transpose), rht_order, rht_seed, rounding, sr_seed,
+                             codes, scales, smma, gs, ws, ws.numel(), stream)
     elif rht:
         nvfp4_rht_quantize_sr(x, rows, cols, x.stride(0), int(transpose), rht_seed, rounding, sr_seed, codes,
                               scales, smma, gs, ws, ws.numel(), stream)
