@@ -72,17 +72,56 @@ def peaks():
 
 # ------------------------------------------------------------------ clocks --
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and clock-event (throttle) reasons sampled during the timed
+    region: NVML read every 10 ms on a thread, the same counters nvidia-smi
+    reports (read only; nothing is set).  Without NVML, nvidia-smi's loop
+    mode.  Only samples taken inside the timed region are kept."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, device=None):
         self.gpu = gpu_index
+        self.device = device
         self.proc = None
         self.lines = []
+        self.samples = []          # (perf_counter, sm MHz, reason mask)
+        self.nvml = None
+        self.handle = None
+        self.max_mhz = None
+        self.running = False
+
+    def _nvml_handle(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        self.nvml = nv
+        if self.device is not None:
+            import torch
+            props = torch.cuda.get_device_properties(self.device)
+            try:
+                return nv.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                pass
+            try:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                return nv.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                pass
+        return nv.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        try:
+            self.handle = self._nvml_handle()
+            nv = self.nvml
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM))
+            self.running = True
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -92,34 +131,57 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while self.running:
+            try:
+                self.samples.append((time.perf_counter(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                     int(get_reasons(h))))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
+            parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                mhz, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
+            self.max_mhz = mx
+            mask = 0
+            for (n, bit), v in zip(self.REASONS[:4], parts[5:9]):
                 if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                    mask |= bit
+            self.samples.append((time.perf_counter(), mhz, mask))
+
+    def stop(self, t_begin: float, t_end: float):
+        if self.nvml is not None:
+            self.running = False
+            self.t.join(timeout=2)
+            src = "nvml"
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+            src = "nvidia-smi"
+        else:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"], "samples": 0}
+        inside = [x for x in self.samples if t_begin <= x[0] <= t_end]
+        sm = [x[1] for x in inside]
+        mask = 0
+        for x in inside:
+            mask |= x[2]
+        reasons = [n for n, bit in self.REASONS if mask & bit]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm), "source": src}
 
 
 # ----------------------------------------------------------- native arm ----
@@ -273,7 +335,7 @@ def native(args):
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ops]
           for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, dev)
     barrier()
     torch.cuda.synchronize()
     clocks.start()
@@ -288,7 +350,7 @@ def native(args):
     wall = time.perf_counter() - wall0
     launches = N.nvfp4_kernel_launches() - launches0
     barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(wall0, wall0 + wall)
     assert N.nvfp4_get_error(s.cuda_stream) == 0
     ms_total = t0.elapsed_time(t1)
     if world > 1:
