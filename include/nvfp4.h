@@ -74,7 +74,8 @@ enum { NVFP4_RNE = 0, NVFP4_SR = 1 };            /* rounding of element codes */
 enum { NVFP4_SCALE_1D = 0, NVFP4_SCALE_2D = 1 };  /* 16 along K | 16x16 tile */
 enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 };   /* GEMM / dequantize output type */
 
-/* Library ABI version (major * 100 + minor). */
+/* Library ABI version (major * 100 + minor): 101 = 1.1, the 1.0 entry points
+ * plus the dual, from-amax, GEMM-amax, MXFP4 and RHT-order ones. */
 int nvfp4_version(void);
 
 /* Human-readable name of a status code (static string, never NULL). */

@@ -40,7 +40,7 @@ nvfp4_status check_quant_common(const void* x, int64_t rows, int64_t cols, int64
 
 extern "C" {
 
-int nvfp4_version(void) { return 100; }
+int nvfp4_version(void) { return 101; }
 
 const char* nvfp4_status_string(nvfp4_status s) {
     switch (s) {

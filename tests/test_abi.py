@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert N.nvfp4_version() >= 100
+    assert N.nvfp4_version() == 101
     for s in range(7):
         assert N.nvfp4_status_string(s)
     assert "unknown" in N.nvfp4_status_string(99)
