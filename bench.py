@@ -418,7 +418,7 @@ def native(args):
         "wall_s_timed": round(wall, 3),
     }
     if not args.no_e2e:
-        result["e2e"] = e2e(torch, N, step, s, args)
+        result["e2e"] = e2e(torch, N, step, s, args, dist if world > 1 else None, world, dev)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         result["cpu_baseline"] = cpu_baseline(target_s=12.0)
     if world > 1:
@@ -443,12 +443,14 @@ def load_traffic():
         return None
 
 
-def e2e(torch, N, step, s, args):
+def e2e(torch, N, step, s, args, dist=None, world=1, dev=None):
     """The same step through the C ABI with host buffers: every step copies its
     inputs in from pinned host memory and its three bf16 results out.  Two
     sets of device buffers let step k compute while the inputs of step k+1
     and the results of step k-1 cross PCIe (one stream each way); the timed
-    region runs from the first copy in to the last copy out."""
+    region runs from the first copy in to the last copy out.  With several
+    ranks (one per GPU, each on its own host buffers) the time is the slowest
+    rank's and the value and byte counts are the whole job's."""
     hx = torch.from_numpy(step.host_np["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
     hw = torch.from_numpy(step.host_np["w"].view(np.int16)).view(torch.bfloat16).pin_memory()
     hdy = torch.from_numpy(step.host_np["dy"].view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -494,6 +496,8 @@ def e2e(torch, N, step, s, args):
     for k in range(2):
         one(k)
     torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
     a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(s_in)
     for k in range(n):
@@ -501,9 +505,11 @@ def e2e(torch, N, step, s, args):
     z.record(s_out)
     torch.cuda.synchronize()
     ms = a.elapsed_time(z) / n
+    if dist is not None:
+        ms = max_over_ranks(ms, dist, dev)
     flops = sum(o[2] for o in step.ops if o[1] == "gemm")
-    return {"value": round(flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": n,
+    return {"value": round(job_tflops(flops, world, ms), 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": int(h2d) * world, "d2h_bytes_per_step": int(d2h) * world, "steps": n,
             "overlap": "step k computes while step k+1's inputs and step k-1's results cross PCIe"}
 
 
