@@ -121,3 +121,20 @@ def test_python_constants_match_header_enums():
     hdr = open(os.path.join(ROOT, "include", "nvfp4.h")).read()
     for name, value in re.findall(r"\b(NVFP4_[A-Z0-9_]+) = (\d+)", hdr):
         assert getattr(N, name) == int(value), name
+
+
+def rhtn(L, **kw):
+    a = dict(x=FAKE, rows=256, cols=64, ld=64, tr=1, order=64, seed=0, rnd=0, sr=0, codes=FAKE, scales=FAKE,
+             mma=None, gs=FAKE, ws=FAKE, wsb=WS)
+    a.update(kw)
+    return L.nvfp4_rht_quantize_n(a["x"], a["rows"], a["cols"], a["ld"], a["tr"], a["order"], a["seed"], a["rnd"],
+                                  a["sr"], a["codes"], a["scales"], a["mma"], a["gs"], a["ws"], a["wsb"], None)
+
+
+def test_rht_quantize_n_validation(L):
+    for order in (0, 8, 48, 256, -16):
+        assert rhtn(L, order=order) == N.NVFP4_ERR_INVALID_ARG, order
+    assert rhtn(L, rows=192, order=128) == N.NVFP4_ERR_UNSUPPORTED_SHAPE      # tokens not a multiple of 128
+    assert rhtn(L, tr=0, rows=32, cols=96, ld=96, order=64) == N.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert rhtn(L, x=None) == N.NVFP4_ERR_INVALID_ARG                            # common checks first
+    assert rhtn(L, x=FAKE + 2) == N.NVFP4_ERR_MISALIGNED
