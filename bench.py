@@ -57,6 +57,9 @@ def parse():
                              "dequantize", "rht_sr", "rht_rne"],
                     help="time one kernel family alone on --shape (profiling mode)")
     ap.add_argument("--shape", default=None, help="M,N,K for gemm; rows,cols otherwise")
+    ap.add_argument("--sweep", action="store_true",
+                    help="quantizer sweep: 2^20 .. 2^30 elements in rows of 4096, three distributions, "
+                         "1D RNE, 2D, RHT + SR row-wise and transposed (one JSON line per case)")
     ap.add_argument("--rht-order", type=int, default=16, choices=[16, 32, 64, 128],
                     help="points of the Hadamard transform for the rht_* ops (rht_t_*: transposed)")
     return ap.parse_args()
@@ -698,9 +701,81 @@ def micro(args):
                       "unit": unit, "note": "profiling mode (one op alone), not a bench line"}), flush=True)
 
 
+def sweep(args):
+    """Quantizer sweep on the device: [R x 4096] bf16 for R = 256, 4096, 65536,
+    262144 (2^20 .. 2^30 elements); values N(0,1), sign * exp(N(0, 2)), or
+    N(0,1) with 0.1% set to +-1e4 (drawn with torch on the device: timing only,
+    not the seeded numpy streams the parity tests use).  Per case the CUDA-event
+    time of each op (both passes), GB/s on the compulsory bytes (one read) and
+    on the bytes moved (two reads), and whether the input fits in L2."""
+    import torch
+    from nvfp4_bit_block_amax_b200 import nvfp4 as N
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    N.lib()
+    hbm = peaks()[0]
+    g = torch.Generator(device=dev)
+    g.manual_seed(4000)
+    s = torch.cuda.Stream(device=dev)
+    C = 4096
+    for dist in ("normal", "lognormal", "outliers"):
+        for R in (256, 4096, 65536, 262144):
+            n = R * C
+            f = torch.randn(R, C, device=dev, generator=g)
+            if dist == "lognormal":
+                sign = torch.where(torch.rand(R, C, device=dev, generator=g) < 0.5, -1.0, 1.0)
+                f = sign * torch.exp(2.0 * f)
+            elif dist == "outliers":
+                k = max(1, round(0.001 * n))
+                idx = torch.randint(0, n, (k,), device=dev, generator=g)
+                f.view(-1)[idx] = torch.where(torch.rand(k, device=dev, generator=g) < 0.5, -1e4, 1e4)
+            x = f.to(torch.bfloat16)
+            del f
+            ws = torch.empty(N.nvfp4_workspace_size(R, C), dtype=torch.uint8, device=dev)
+            gs = torch.empty(1, dtype=torch.float32, device=dev)
+            cr = torch.empty(R, C // 2, dtype=torch.uint8, device=dev)
+            ct = torch.empty(C, R // 2, dtype=torch.uint8, device=dev)
+            mr = torch.empty(N.nvfp4_mma_scale_bytes(R, C), dtype=torch.uint8, device=dev)
+            mt = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)
+            q1 = 2 + 0.5 + 1 / 16
+            q2 = 2 + 0.5 + 0.5 + 2 / 16
+            cases = [
+                ("1d_rne", lambda: N.nvfp4_quantize_1d(x, R, C, C, 0, N.NVFP4_RNE, 0, cr, None, mr, gs, ws,
+                                                       ws.numel(), s), q1),
+                ("2d_rne", lambda: N.nvfp4_quantize_2d(x, R, C, C, cr, ct, None, mr, mt, gs, ws, ws.numel(), s), q2),
+                ("rht_sr_rowwise", lambda: N.nvfp4_rht_quantize_sr(x, R, C, C, 0, 5, N.NVFP4_SR, 6, cr, None, mr, gs,
+                                                                   ws, ws.numel(), s), q1),
+                ("rht_sr_transposed", lambda: N.nvfp4_rht_quantize_sr(x, R, C, C, 1, 5, N.NVFP4_SR, 6, ct, None, mt,
+                                                                      gs, ws, ws.numel(), s), q1),
+            ]
+            for name, fn, per in cases:
+                steps = 20 if n >= (1 << 28) else 100
+                for _ in range(3):
+                    fn()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s)
+                for _ in range(steps):
+                    fn()
+                e1.record(s)
+                torch.cuda.synchronize()
+                assert N.nvfp4_get_error(s.cuda_stream) == 0
+                ms = e0.elapsed_time(e1) / steps
+                comp = n * per / (ms * 1e-3) / 1e9
+                moved = n * (per + 2) / (ms * 1e-3) / 1e9
+                print(json.dumps({"sweep": name, "dist": dist, "rows": R, "cols": C, "elements": n,
+                                  "ms": round(ms, 4), "gbs_compulsory": round(comp, 1),
+                                  "gbs_moved": round(moved, 1), "frac_hbm_moved": round(moved / hbm, 3),
+                                  "l2_resident": n * 2 < 126e6}), flush=True)
+            del x, cr, ct, mr, mt
+            torch.cuda.empty_cache()
+
+
 if __name__ == "__main__":
     a = parse()
-    if a.op:
+    if a.sweep:
+        sweep(a)
+    elif a.op:
         micro(a)
     elif a.impl == "reference":
         reference(a)
