@@ -243,20 +243,25 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
     const int64_t total = p.rows * upr;
     const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
     const int64_t wid = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    const int64_t per = (total + nwarps - 1) / nwarps;
-    int64_t u = wid * per;
-    const int64_t uend = min(total, u + per);
+    // Groups of U consecutive units, interleaved over the warps (group g goes
+    // to warp g mod nwarps): at any moment the grid works on a narrow window of
+    // the tensor, which keeps the address translations it needs few.
+    constexpr int U = 2;
+    const int64_t step = nwarps * U;                   // units between a warp's groups
+    const int64_t step_rows = step / upr, step_uc = step - step_rows * upr;
+    int64_t u = wid * U;
+    const int64_t uend = total;
     const int64_t kb = p.cols >> 4;
     const bool a32 = ((reinterpret_cast<uintptr_t>(p.x) & 31u) == 0) && ((p.ld & 15) == 0);
     uint32_t amax_bits = 0;
-    constexpr int U = 2;
     if (u < uend) {
-        int64_t row = u / upr;
-        int64_t uc = u - row * upr;
-        for (; u < uend; u += U) {
+        int64_t row0 = u / upr;
+        int64_t uc0 = u - row0 * upr;
+        for (; u < uend; u += step) {
             uint32_t w[U][8];
             int64_t rr[U], cc[U];
             bool ok[U];
+            int64_t row = row0, uc = uc0;
 #pragma unroll
             for (int k = 0; k < U; ++k) {
                 rr[k] = row;
@@ -272,6 +277,13 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
                     uc = 0;
                     ++row;
                 }
+            }
+            // the next group of this warp
+            row0 += step_rows;
+            uc0 += step_uc;
+            if (uc0 >= upr) {
+                uc0 -= upr;
+                ++row0;
             }
 #pragma unroll
             for (int k = 0; k < U; ++k) {
