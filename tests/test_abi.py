@@ -138,3 +138,43 @@ def test_rht_quantize_n_validation(L):
     assert rhtn(L, tr=0, rows=32, cols=96, ld=96, order=64) == N.NVFP4_ERR_UNSUPPORTED_SHAPE
     assert rhtn(L, x=None) == N.NVFP4_ERR_INVALID_ARG                            # common checks first
     assert rhtn(L, x=FAKE + 2) == N.NVFP4_ERR_MISALIGNED
+
+
+def test_dual_from_amax_and_gemm_amax_validation(L):
+    d = lambda **kw: L.nvfp4_quantize_dual(
+        kw.get("x", FAKE), 32, 64, 64, kw.get("rnd", 1), 0, FAKE, FAKE, None, FAKE, 5, 6, kw.get("ct", FAKE), FAKE,
+        None, kw.get("gt", FAKE), FAKE, kw.get("wsb", WS), None)
+    assert d(x=None) == N.NVFP4_ERR_INVALID_ARG
+    assert d(ct=None) == N.NVFP4_ERR_INVALID_ARG             # the transposed half is checked too
+    assert d(gt=None) == N.NVFP4_ERR_INVALID_ARG
+    assert d(rnd=3) == N.NVFP4_ERR_INVALID_ARG
+    assert d(ct=FAKE + 4) == N.NVFP4_ERR_MISALIGNED
+    assert d() == N.NVFP4_ERR_WORKSPACE                       # one workspace's worth is not enough for two
+    q = lambda **kw: L.nvfp4_quantize_1d_from_amax(FAKE, 32, 64, 64, 0, 0, 0, kw.get("amax", FAKE), FAKE, FAKE,
+                                                   None, FAKE, None)
+    assert q(amax=None) == N.NVFP4_ERR_INVALID_ARG and q(amax=FAKE + 2) == N.NVFP4_ERR_MISALIGNED
+    w = lambda **kw: L.nvfp4_quantize_2d_from_amax(FAKE, 32, 64, 64, kw.get("amax", FAKE), FAKE, None, FAKE, None,
+                                                   None, FAKE, None)
+    assert w(amax=None) == N.NVFP4_ERR_INVALID_ARG and w(amax=FAKE + 2) == N.NVFP4_ERR_MISALIGNED
+    g = lambda **kw: L.nvfp4_gemm_amax(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 128, kw.get("K", 256), 1, FAKE, 128,
+                                       kw.get("amax", FAKE), None)
+    assert g(amax=None) == N.NVFP4_ERR_INVALID_ARG and g(amax=FAKE + 2) == N.NVFP4_ERR_MISALIGNED
+    assert g(K=96) == N.NVFP4_ERR_UNSUPPORTED_SHAPE
+
+
+def test_mxfp4_and_selftest_validation(L):
+    assert L.nvfp4_mxfp4_quantize(FAKE, 4, 48, 48, FAKE, FAKE, None, None) == N.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_mxfp4_quantize(None, 4, 64, 64, FAKE, FAKE, None, None) == N.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_mxfp4_quantize(FAKE, 4, 64, 64, FAKE, None, None, None) == N.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_mxfp4_quantize(FAKE, 4, 64, 64, FAKE + 8, FAKE, None, None) == N.NVFP4_ERR_MISALIGNED
+    assert L.nvfp4_mxfp4_dequantize(FAKE, FAKE, 4, 64, 9, FAKE, None) == N.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_mxfp4_dequantize(FAKE, FAKE, 4, 40, 0, FAKE, None) == N.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_mxfp4_gemm(FAKE, FAKE, FAKE, FAKE, 128, 128, 96, 1, FAKE, 128, None) == \
+        N.NVFP4_ERR_UNSUPPORTED_SHAPE
+    assert L.nvfp4_mxfp4_gemm(None, FAKE, FAKE, FAKE, 128, 128, 256, 1, FAKE, 128, None) == N.NVFP4_ERR_INVALID_ARG
+    for limit in (0, 999, 2000000001):
+        assert L.nvfp4_selftest_wait_timeout(limit, None) == N.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_quantize_1d_noalloc(None, 32, 64, 64, 0, 0, 0, FAKE, FAKE, None, FAKE, None) == \
+        N.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_quantize_1d_noalloc(FAKE, 32, 40, 40, 0, 0, 0, FAKE, FAKE, None, FAKE, None) == \
+        N.NVFP4_ERR_UNSUPPORTED_SHAPE
