@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-chain", action="store_true", help="skip the chained-layer measurement (amax from the GEMM)")
     ap.add_argument("--op", default=None,
                     choices=["gemm", "gemm_amax", "quantize_1d", "quantize_1d_sr", "quantize_2d", "rht_t_sr",
                              "rht_t_rne", "quantize_1d_from_amax", "quantize_2d_from_amax", "mx_quantize",
@@ -420,6 +421,8 @@ def native(args):
         "gpu_launches": int(launches),
         "wall_s_timed": round(wall, 3),
     }
+    if not args.no_chain:
+        result["chain"] = chain(torch, N, G, step, s, args)
     if not args.no_e2e:
         result["e2e"] = e2e(torch, N, step, s, args, dist if world > 1 else None, world, dev)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
@@ -429,6 +432,73 @@ def native(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def chain(torch, N, G, step, s, args):
+    """Two chained layers with the amax handed over by its producer ("NVFP4
+    Is a Scaling System", "Where speed and accuracy claims can fail":
+    quantization and scale handling cost work): Y = X . W1^T by the GEMM that
+    also writes max |Y| (nvfp4_gemm_amax), Y quantized in one read from that
+    amax (nvfp4_quantize_1d_from_amax), then Z = Yq . W2^T, W2 [hidden x ffn]
+    2D-quantized outside the timed region.  Beside it, the two-pass
+    quantize of the same Y (amax pass + encode), for the comparison.  X and W1
+    are the step's quantized operands."""
+    t, h, f = T, H, F
+    dev = step.dev
+    cs = s.cuda_stream
+    w2 = torch.from_numpy(G.weight(h, f, G.seeds("mlp_step")[0] + 3).view(np.int16)).view(torch.bfloat16).to(dev)
+    e = lambda *sh: torch.empty(*sh, dtype=torch.uint8, device=dev)
+    mb = N.nvfp4_mma_scale_bytes
+    g = torch.zeros(8, dtype=torch.float32, device=dev)
+    w2q = (e(h, f // 2), e(mb(h, f)))
+    N.nvfp4_quantize_2d(w2, h, f, f, w2q[0], None, None, w2q[1], None, g[0:1], step.ws, step.ws.numel(), cs)
+    del w2
+    yq, yq2 = (e(t, f // 2), e(mb(t, f))), (e(t, f // 2), e(mb(t, f)))
+    z = torch.empty(t, h, dtype=torch.bfloat16, device=dev)
+    y, amax = step.y, g[1:2]
+    ops = [
+        lambda: N.nvfp4_gemm_amax(step.xq[0], step.xq[1], step.gp[0], step.wq[0], step.wq[1], step.gp[1], t, f, h,
+                                  N.NVFP4_OUT_BF16, y, f, amax, cs),
+        lambda: N.nvfp4_quantize_1d_from_amax(y, t, f, f, 0, N.NVFP4_RNE, 0, amax, yq[0], None, yq[1], g[2:3], cs),
+        lambda: N.nvfp4_gemm(yq[0], yq[1], g[2:3], w2q[0], w2q[1], g[0:1], t, h, f, N.NVFP4_OUT_BF16, z, h, cs),
+        lambda: N.nvfp4_quantize_1d(y, t, f, f, 0, N.NVFP4_RNE, 0, yq2[0], None, yq2[1], g[3:4], step.ws,
+                                    step.ws.numel(), cs),
+    ]
+    names = ["gemm_amax up (Y = X W1^T, + max|Y|)", "quantize_1d_from_amax Y (one read)", "gemm down (Z = Yq W2^T)",
+             "quantize_1d Y two-pass (comparison, not in the chain)"]
+    for _ in range(max(args.warmup, 1)):
+        for op in ops:
+            op()
+    torch.cuda.synchronize()
+    n = max(args.steps, 3)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ops] for _ in range(n)]
+    for k in range(n):
+        for i, op in enumerate(ops):
+            ev[k][i][0].record(s)
+            op()
+            ev[k][i][1].record(s)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error(cs) == 0
+    same = bool(torch.equal(yq[0], yq2[0]) and torch.equal(yq[1], yq2[1]) and torch.equal(g[2], g[3]))
+    ms = [statistics.mean(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(n)) for i in range(len(ops))]
+    hbm = peaks()[0]
+    elems = t * f
+    comp = elems * (2 + 0.5 + 1 / 16)
+    moved2 = elems * (2 + 2 + 0.5 + 1 / 16)
+    chain_ms = ms[0] + ms[1] + ms[2]
+    flops = 2 * 2.0 * t * f * h
+    return {"workload": f"X [{t} x {h}] -> Y = X W1^T [{t} x {f}] bf16 -> Yq (1D RNE) -> Z = Yq W2^T [{t} x {h}] bf16",
+            "steps": n, "ms_per_chain": round(chain_ms, 4), "tflops": round(flops / (chain_ms * 1e-3) / 1e12, 1),
+            "ops": [{"op": nm, "ms": round(m, 4)} for nm, m in zip(names, ms)],
+            "quantize_single_read": {"ms": round(ms[1], 4), "gbs": round(comp / (ms[1] * 1e-3) / 1e9, 1),
+                                     "frac_hbm": round(comp / (ms[1] * 1e-3) / 1e9 / hbm, 4),
+                                     "bytes_per_elem": 2.5625},
+            "quantize_two_pass": {"ms": round(ms[3], 4), "gbs_moved": round(moved2 / (ms[3] * 1e-3) / 1e9, 1),
+                                  "frac_hbm_moved": round(moved2 / (ms[3] * 1e-3) / 1e9 / hbm, 4),
+                                  "gbs_compulsory": round(comp / (ms[3] * 1e-3) / 1e9, 1),
+                                  "frac_hbm_compulsory": round(comp / (ms[3] * 1e-3) / 1e9 / hbm, 4),
+                                  "bytes_per_elem_moved": 4.5625},
+            "single_read_equals_two_pass": same}
 
 
 def load_traffic():
@@ -554,7 +624,78 @@ def blas_threads():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 SAMPLE = (512, 1024, 2048)   # tokens, hidden, ffn of the oracle's sample of the step
+QSAMPLE = (1024, 8192)       # rows, cols of the quantizer oracle's sample (rows of the step's activation recipe)
+
+
+_QX = {}
+
+
+def _oracle_sample(rows, cols):
+    from nvfp4_bit_block_amax_b200 import inputs as G
+    if (rows, cols) not in _QX:
+        _QX[(rows, cols)] = G.activation(rows, cols, G.seeds("mlp_step")[0])
+    return _QX[(rows, cols)]
+
+
+def _oracle_rows_worker(args):
+    """One process of the multi-core quantizer oracle on Q rows [r0, r1) of
+    the sample: the amax of those rows (sg is None), or their codes given the
+    global scale sg (spawned, no GPU)."""
+    r0, r1, rows, cols, sg = args
+    from oracle import oracle as O
+    x = _oracle_sample(rows, cols)
+    if sg is None:
+        return O.amax(x[r0:r1])
+    O.quantize_1d_rows(x, sg, range(r0, r1))
+    return 0.0
+
+
+def quantizer_oracle_rates(procs=None):
+    """The scalar C quantizer (1D RNE: amax pass, then encode) on a [1024 x
+    8192] sample of the step's activation recipe: GB/s of compulsory bytes
+    (2.5625 per element) on one thread, and with the rows split over a
+    process pool on every host core (both passes; spawn start, so no fork
+    after CUDA)."""
+    import multiprocessing as mp
+    from oracle import oracle as O
+    rows, cols = QSAMPLE
+    x = _oracle_sample(rows, cols)
+    O.lib()
+    t0 = time.perf_counter()
+    sg = O.global_scale(O.amax(x))
+    O.quantize_1d_rows(x, sg, range(rows))
+    t1 = time.perf_counter() - t0
+    nbytes = rows * cols * (2 + 0.5 + 1 / 16)
+    procs = procs or os.cpu_count() or 1
+    ctx = mp.get_context("spawn")
+    step = (rows + procs - 1) // procs
+    ranges = [(r, min(rows, r + step)) for r in range(0, rows, step)]
+    with ctx.Pool(len(ranges)) as pool:
+        pool.map(_oracle_rows_worker, [(a, b, rows, cols, None) for a, b in ranges])   # warm: imports, sample
+        t0 = time.perf_counter()
+        amax = max(pool.map(_oracle_rows_worker, [(a, b, rows, cols, None) for a, b in ranges]))
+        sg_n = O.global_scale(amax)
+        pool.map(_oracle_rows_worker, [(a, b, rows, cols, sg_n) for a, b in ranges])
+        tn = time.perf_counter() - t0
+    assert sg_n == sg
+    return {"sample": f"1D RNE quantize of a [{rows} x {cols}] bf16 activation (amax pass + encode, "
+                      f"{nbytes / 1e6:.1f} MB compulsory)",
+            "gbs_1_thread": round(nbytes / t1 / 1e9, 4), "gbs_all_cores": round(nbytes / tn / 1e9, 4),
+            "processes": len(ranges)}
 
 
 def cpu_baseline(target_s=12.0):
@@ -565,17 +706,31 @@ def cpu_baseline(target_s=12.0):
         secs += dt
         flops += fl
         n += 1
-    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{n} oracle passes of the step at tokens {t}, hidden {h}, ffn {f} (same recipes); scalar C "
-                      "quantizers on 1 thread, float64 BLAS GEMMs", "seconds": round(secs, 2)}
+    blas = blas_threads()
+    out = {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": blas, "kind": "oracle",
+           "sample": f"{n} oracle passes of the step at tokens {t}, hidden {h}, ffn {f} (same recipes); scalar C "
+                     "quantizers on 1 thread, float64 BLAS GEMMs", "seconds": round(secs, 2),
+           "threads": {"quantizers": 1, "blas_gemm": blas}, "host_cores": os.cpu_count(), "cpu_model": cpu_model()}
+    try:
+        out["quantizer_oracle"] = quantizer_oracle_rates()
+    except Exception as e:   # the pool is a report, not part of the contract
+        out["quantizer_oracle"] = {"error": repr(e)[:200]}
+    return out
+
+
+REF_SAMPLE = (256, 512, 1024)   # tokens, hidden, ffn of each step of the reference arm
 
 
 def reference(args):
+    """The oracle as the reference arm: each step is the whole MLP step at
+    tokens 256, hidden 512, ffn 1024 (a bounded sample of the bench's
+    workload, same recipes), on the host cores.  The line names that sample;
+    its value is the sample's throughput, not the full step's."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    t, h, f = 256, 512, 1024
+    t, h, f = REF_SAMPLE
     for _ in range(args.warmup):
         oracle_step(t, h, f)
     secs, flops = 0.0, 0.0
@@ -584,13 +739,18 @@ def reference(args):
         secs += dt
         flops += fl
     v = flops / secs / 1e12
+    blas = blas_threads()
+    sample = (f"each step: the whole MLP step (quantize X 1D RNE, W 2D, dY 1D SR, RHT dY^T SR / X^T RNE; three "
+              f"float64 GEMMs) at tokens {t}, hidden {h}, ffn {f} -- a sample of {WORKLOAD}")
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 quantizers, f64 GEMM",
             "data": "synthetic (same seeded recipes)",
-            "config": {"workload": WORKLOAD, "tokens": T, "hidden": H, "ffn": F, "parallelism": "oracle on host"},
-            "cpu_baseline": {"kind": "oracle", "cores": blas_threads(), "value": round(v, 6), "unit": "TFLOP/s",
-                             "sample": f"each step: the whole step at tokens {t}, hidden {h}, ffn {f}"},
+            "config": {"workload": WORKLOAD, "sample_of_workload": True, "tokens": t, "hidden": h, "ffn": f,
+                       "parallelism": "oracle on host"},
+            "cpu_baseline": {"kind": "oracle", "cores": blas, "value": round(v, 6), "unit": "TFLOP/s",
+                             "sample": sample, "threads": {"quantizers": 1, "blas_gemm": blas},
+                             "host_cores": os.cpu_count(), "cpu_model": cpu_model()},
             "e2e": {"value": round(v, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

@@ -130,13 +130,20 @@ nvfp4_status nvfp4_quantize_1d(const void* x, int64_t rows, int64_t cols, int64_
  * amax scratch (one partial maximum per CTA of the amax pass) is a static
  * 4 KiB array inside the library (1024 partials), which every GPU that loads
  * the library holds until the process exits.
- *   - The first call on a device looks up that array's device address (once
- *     per device, with that device current); make this first call before any
- *     stream capture.
+ *   - The first call on a device looks up that array's device address (with
+ *     that device current) and keeps it for later calls; make this first
+ *     call before any stream capture.  The address belongs to the CUDA
+ *     context current at the lookup: when a call finds another context
+ *     current (after cudaDeviceReset, or once the primary context was
+ *     released and created again), it looks the address up again, so a
+ *     context reset leaves no stale address behind; the first call after the
+ *     reset is again a set-up call.
  *   - The amax pass launches at most 4 CTAs per SM, one partial each; on a
  *     device with more than 256 SMs a call that would need more than 1024
  *     partials is refused with NVFP4_ERR_WORKSPACE before anything is
- *     enqueued.
+ *     enqueued (the environment variable NVFP4_SM_COUNT, a positive integer,
+ *     replaces the device's SM count in all grid sizing of the quantizers;
+ *     results do not depend on it, this capacity check does).
  *   - All calls on a device share the array, which keeps the last call's
  *     contents; each call's amax pass overwrites every entry its encode pass
  *     reads, so nothing needs clearing between calls.  Calls that overlap on
@@ -260,7 +267,12 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int s
  * the matmuls; "Hardware support still needs a full sentence" -- native
  * block-scaled matrix operations on Blackwell tensor cores]:
  *   C[i][j] = alpha * sum_k (a_ik * sa_i,k/16) * (b_jk * sb_j,k/16),
- *   alpha = RN(s_global_A * s_global_B), accumulated in FP32 in tensor memory.
+ *   the sum accumulated in FP32 in tensor memory, then C = RN(sum * alpha)
+ *   with alpha = RN(s_global_A * s_global_B).  When that alpha is not a
+ *   normal binary32 number (both global scales tiny, product subnormal or
+ *   zero; or both huge, product overflowing), the scales are applied one
+ *   after the other, C = RN(RN(sum * s_global_A) * s_global_B), so that C
+ *   keeps its precision wherever C itself is a normal number.
  *   a_codes [M x K/2], a_scales_mma (MMA layout, R = M), a_gs device float;
  *   b_codes [N x K/2], b_scales_mma (MMA layout, R = N), b_gs device float;
  *   c [M x ldc] FP32 or bf16 (row-major), ldc >= N.

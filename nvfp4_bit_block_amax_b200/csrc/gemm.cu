@@ -329,6 +329,26 @@ __device__ __forceinline__ uint32_t packed_row_amax(const uint32_t (&packed)[64]
     return absmax2_fold(acc);
 }
 
+// Output scale factors (a1, a2): C = RN(RN(acc * a1) * a2).  Normally a1 =
+// alpha = RN(s_global_A * s_global_B) and a2 = 1 (the second multiply is
+// exact).  When alpha is not a normal binary32 number -- both global scales
+// tiny, so that their product is subnormal or zero, or both huge, so that it
+// overflows -- the two global scales are applied one after the other
+// (a1 = s_global_A, a2 = s_global_B): the accumulator times one scale stays
+// in range wherever C itself does.  MXFP4 operands have no global scale.
+__device__ __forceinline__ float2 out_scales(const KParams& p) {
+    if (!p.a_gs) return make_float2(1.0f, 1.0f);
+    const float sa = __ldg(p.a_gs), sb = __ldg(p.b_gs);
+    const float alpha = __fmul_rn(sa, sb);
+    if (alpha >= 0x1p-126f && alpha <= 0x1.fffffep127f) return make_float2(alpha, 1.0f);
+    return make_float2(sa, sb);
+}
+// Two accumulator values scaled by (a1, a2), in f32x2 multiplies.
+__device__ __forceinline__ float2 scale_out2(uint32_t u0, uint32_t u1, float2 al) {
+    const float2 v = __fmul2_rn(make_float2(__uint_as_float(u0), __uint_as_float(u1)), make_float2(al.x, al.x));
+    return __fmul2_rn(v, make_float2(al.y, al.y));
+}
+
 // Tile t -> (tm, tn).  Tiles are taken in groups of group_m M-tiles; inside a
 // group M runs fastest, then N.  The CTAs working at the same time then share
 // group_m A panels and a few B panels, which stay resident in L2.
@@ -347,7 +367,7 @@ __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& tm, in
 // pairs, 64 registers), arrive on tmem_empty, then store.  False when the
 // bounded wait for the accumulator ran out.
 __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int half, int q, int lane, uint32_t tmem,
-                                              float alpha, uint32_t bar_tfull, uint32_t bar_tempty,
+                                              float2 alpha, uint32_t bar_tfull, uint32_t bar_tempty,
                                               uint32_t& acc_phase, volatile int* abort_flag, uint32_t& amax_acc) {
     if (!mbar_wait(bar_tfull, acc_phase, abort_flag)) return false;
     tc_fence_after();
@@ -370,10 +390,10 @@ __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int ha
             tc_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                const __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v0[2 * e]), alpha),
-                                                                __fmul_rn(__uint_as_float(v0[2 * e + 1]), alpha));
-                const __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v1[2 * e]), alpha),
-                                                                __fmul_rn(__uint_as_float(v1[2 * e + 1]), alpha));
+                const float2 f0 = scale_out2(v0[2 * e], v0[2 * e + 1], alpha);
+                const float2 f1 = scale_out2(v1[2 * e], v1[2 * e + 1], alpha);
+                const __nv_bfloat162 h0 = __floats2bfloat162_rn(f0.x, f0.y);
+                const __nv_bfloat162 h1 = __floats2bfloat162_rn(f1.x, f1.y);
                 packed[32 * i + e] = *reinterpret_cast<const uint32_t*>(&h0);
                 packed[32 * i + 16 + e] = *reinterpret_cast<const uint32_t*>(&h1);
             }
@@ -410,10 +430,9 @@ __device__ __forceinline__ bool epilogue_half(const KParams& p, int tile, int ha
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
                     const int cc = 32 * i + 4 * g;
-                    const float4 f = make_float4(__fmul_rn(__uint_as_float(v[4 * g]), alpha),
-                                                 __fmul_rn(__uint_as_float(v[4 * g + 1]), alpha),
-                                                 __fmul_rn(__uint_as_float(v[4 * g + 2]), alpha),
-                                                 __fmul_rn(__uint_as_float(v[4 * g + 3]), alpha));
+                    const float2 f01 = scale_out2(v[4 * g], v[4 * g + 1], alpha);
+                    const float2 f23 = scale_out2(v[4 * g + 2], v[4 * g + 3], alpha);
+                    const float4 f = make_float4(f01.x, f01.y, f23.x, f23.y);
                     if (cc + 4 <= ncols) {
                         *reinterpret_cast<float4*>(crow + cc) = f;
                         fmax = fmaxf(fmaxf(fmaxf(fmax, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
@@ -567,7 +586,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         // the 16 bytes at offset 16 l of the step's 512-byte scale chunks.
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float alpha = p.a_gs ? __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs)) : 1.0f;
+        const float2 alpha = out_scales(p);
         int s = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
@@ -643,7 +662,7 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     } else {
         // ---------------------------------------- epilogue, columns 128..255 ----
         const int q = warp & 3;
-        const float alpha = p.a_gs ? __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs)) : 1.0f;
+        const float2 alpha = out_scales(p);
         uint32_t acc_phase = 0;
         uint32_t amax_acc = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x)
@@ -688,7 +707,7 @@ constexpr int P_SMEM_BYTES = P_OFF_MISC + 16 + 1024;
 constexpr uint32_t kIdescPair = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 
 __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, int half, int q, int lane, uint32_t rank,
-                                                   uint32_t tmem, float alpha, uint32_t bar_tfull, uint32_t bar_tempty,
+                                                   uint32_t tmem, float2 alpha, uint32_t bar_tfull, uint32_t bar_tempty,
                                                    uint32_t& acc_phase, volatile int* abort_flag, uint32_t& amax_acc) {
     if (!mbar_wait_cluster(bar_tfull, acc_phase, abort_flag)) return false;
     tc_fence_after();
@@ -717,10 +736,10 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
             tc_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                const __nv_bfloat162 h0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v0[2 * e]), alpha),
-                                                                __fmul_rn(__uint_as_float(v0[2 * e + 1]), alpha));
-                const __nv_bfloat162 h1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v1[2 * e]), alpha),
-                                                                __fmul_rn(__uint_as_float(v1[2 * e + 1]), alpha));
+                const float2 f0 = scale_out2(v0[2 * e], v0[2 * e + 1], alpha);
+                const float2 f1 = scale_out2(v1[2 * e], v1[2 * e + 1], alpha);
+                const __nv_bfloat162 h0 = __floats2bfloat162_rn(f0.x, f0.y);
+                const __nv_bfloat162 h1 = __floats2bfloat162_rn(f1.x, f1.y);
                 packed[32 * i + e] = *reinterpret_cast<const uint32_t*>(&h0);
                 packed[32 * i + 16 + e] = *reinterpret_cast<const uint32_t*>(&h1);
             }
@@ -754,10 +773,9 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
                     const int cc = 32 * i + 4 * g;
-                    const float4 f = make_float4(__fmul_rn(__uint_as_float(v[4 * g]), alpha),
-                                                 __fmul_rn(__uint_as_float(v[4 * g + 1]), alpha),
-                                                 __fmul_rn(__uint_as_float(v[4 * g + 2]), alpha),
-                                                 __fmul_rn(__uint_as_float(v[4 * g + 3]), alpha));
+                    const float2 f01 = scale_out2(v[4 * g], v[4 * g + 1], alpha);
+                    const float2 f23 = scale_out2(v[4 * g + 2], v[4 * g + 3], alpha);
+                    const float4 f = make_float4(f01.x, f01.y, f23.x, f23.y);
                     if (cc + 4 <= ncols) {
                         *reinterpret_cast<float4*>(crow + cc) = f;
                         fmax = fmaxf(fmaxf(fmaxf(fmax, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
@@ -906,7 +924,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
         // ------------------------------- scales -> TMEM, and the epilogue ----
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float alpha = p.a_gs ? __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs)) : 1.0f;
+        const float2 alpha = out_scales(p);
         int s = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
@@ -981,7 +999,7 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
     } else {
         // ---------------------------------------- epilogue, columns 128..255 ----
         const int q = warp & 3;
-        const float alpha = p.a_gs ? __fmul_rn(__ldg(p.a_gs), __ldg(p.b_gs)) : 1.0f;
+        const float2 alpha = out_scales(p);
         uint32_t acc_phase = 0;
         uint32_t amax_acc = 0;
         for (int tile = cluster; tile < num_tiles; tile += n_clusters)

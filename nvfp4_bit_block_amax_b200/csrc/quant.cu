@@ -12,10 +12,14 @@
 //                   codes (RNE or stochastic rounding), packed two per byte.
 // All floating-point steps are single IEEE binary32 operations in the order
 // stated in nvfp4.h (this file is built with --fmad=false).
+#include <cuda.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 #include <algorithm>
+#include <atomic>
+#include <cstdlib>
 #include <mutex>
 
 namespace nvfp4 {
@@ -25,17 +29,26 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
 
+// SM count of the current device, cached per device.  NVFP4_SM_COUNT, when
+// set to a positive integer, replaces it in the grid sizing (the kernels'
+// results do not depend on the grid; the allocation-free entry point's
+// capacity check does, which is how that check is exercised without a GPU).
 int sm_count() {
-    static int cached[64] = {0};
+    if (const char* o = getenv("NVFP4_SM_COUNT")) {
+        const int n = atoi(o);
+        if (n > 0) return n;
+    }
+    static std::atomic<int> cached[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
-    if (!cached[dev]) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (!n) {
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cached[dev] = n > 0 ? n : 148;
+        if (n <= 0) n = 148;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 // ------------------------------------------------------------ amax (plain) --
@@ -966,24 +979,62 @@ constexpr int kNoAllocPartials = 1024;   // 4 KiB
 static __device__ __align__(256) uint32_t g_noalloc_partials[kNoAllocPartials];
 
 namespace {
-std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[64] = {nullptr};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of the static scratch on the current device, looked up once
-// per device (host code only sees a stand-in symbol, never a device address).
+// Identity of the CUDA context current on this thread (0 when none is, or
+// when the driver cannot tell).  A context that is destroyed and created
+// again (cudaDeviceReset, a primary context released and retained) gets a
+// new identity, and the library's device image -- the scratch array with it
+// -- may then sit at another address.
+unsigned long long current_context_id() {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(f);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+std::mutex g_noalloc_mutex;
+struct ScratchSlot {
+    unsigned long long ctx_id;
+    void* ptr;
+};
+ScratchSlot g_noalloc_slot[64] = {};
+
+// Device address of the static scratch in the current context (host code
+// only sees a stand-in symbol, never a device address).  Looked up with the
+// device current the first time a context uses it, and again whenever the
+// current context is not the one the cached address belongs to.
 cudaError_t noalloc_scratch(uint32_t** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    ScratchSlot& slot = g_noalloc_slot[dev];
+    const unsigned long long id = current_context_id();
+    if (!slot.ptr || id == 0 || id != slot.ctx_id) {
         void* ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_noalloc_partials);
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_partials);   // also makes the device's context current
         if (e != cudaSuccess) return e;
-        g_noalloc_ptr[dev] = ptr;
+        slot.ptr = ptr;
+        slot.ctx_id = current_context_id();
     }
-    *out = static_cast<uint32_t*>(g_noalloc_ptr[dev]);
+    *out = static_cast<uint32_t*>(slot.ptr);
     return cudaSuccess;
 }
 }  // namespace
@@ -996,14 +1047,14 @@ int noalloc_capacity() { return kNoAllocPartials; }
 // refused (*too_big = true) before anything is enqueued.
 cudaError_t launch_quantize_1d_noalloc(const QuantArgs& a, cudaStream_t s, int* launches, bool* too_big) {
     *too_big = false;
-    uint32_t* scratch = nullptr;
-    cudaError_t e = noalloc_scratch(&scratch);
-    if (e != cudaSuccess) return e;
     const int g = plain_amax_grid(a.rows, a.cols);
     if (g > kNoAllocPartials) {
         *too_big = true;
         return cudaSuccess;
     }
+    uint32_t* scratch = nullptr;
+    cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return e;
     QuantArgs b = a;
     b.rht = 0;
     b.given_amax = nullptr;

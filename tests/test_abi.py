@@ -178,3 +178,24 @@ def test_mxfp4_and_selftest_validation(L):
         N.NVFP4_ERR_INVALID_ARG
     assert L.nvfp4_quantize_1d_noalloc(FAKE, 32, 40, 40, 0, 0, 0, FAKE, FAKE, None, FAKE, None) == \
         N.NVFP4_ERR_UNSUPPORTED_SHAPE
+
+
+def test_noalloc_refuses_a_grid_beyond_its_scratch(L, monkeypatch):
+    """The allocation-free quantizer holds 1024 amax partials; its amax pass
+    takes up to 4 CTAs per SM.  With the SM count overridden to 300 a large
+    tensor would need 1200 partials: the call must say NVFP4_ERR_WORKSPACE,
+    enqueue nothing and leave its outputs untouched.  The outputs here are
+    host buffers standing in for device ones (nothing may write them); the
+    refusal happens before any CUDA call, so no GPU is needed."""
+    import numpy as np
+    rows, cols = 4096, 4096                   # 2M 16-byte vectors: 2048 CTAs wanted
+    codes = np.full(rows * cols // 2 + 64, 0xAB, dtype=np.uint8)
+    scales = np.full(rows * cols // 16 + 64, 0xAB, dtype=np.uint8)
+    gs = np.full(16, 0xAB, dtype=np.uint8)
+    al = lambda a: (a.ctypes.data + 15) & ~15
+    before = L.nvfp4_kernel_launches()
+    monkeypatch.setenv("NVFP4_SM_COUNT", "300")
+    st = L.nvfp4_quantize_1d_noalloc(FAKE, rows, cols, cols, 0, 0, 0, al(codes), al(scales), None, al(gs), None)
+    assert st == N.NVFP4_ERR_WORKSPACE
+    assert L.nvfp4_kernel_launches() == before
+    assert (codes == 0xAB).all() and (scales == 0xAB).all() and (gs == 0xAB).all()

@@ -9,7 +9,7 @@ import torch
 from nvfp4_bit_block_amax_b200 import inputs as G
 from nvfp4_bit_block_amax_b200 import nvfp4 as N
 from oracle import oracle as O
-from tests.helpers import mma_layout, to_device_bf16
+from tests.helpers import mma_layout, to_device_bf16, unpack_codes
 
 pytestmark = pytest.mark.gpu
 
@@ -132,11 +132,50 @@ def test_quantizer_sweep(n, dist):
     torch.cuda.synchronize()
     check_quantized_rows(q3, x, rows, rht=True, rht_seed=seed + 100, rounding=1, sr_seed=seed + 101)
     del q3
-    if n <= (1 << 24):
+    if n <= (1 << 28):
         q4 = N.quantize_1d(xd, transpose=True, rht=True, rht_seed=seed + 100, rounding=N.NVFP4_SR, sr_seed=seed + 102)
         torch.cuda.synchronize()
         check_quantized_rows(q4, x, sample_rows(cols, 6, seed=3), transpose=True, rht=True, rht_seed=seed + 100,
                              rounding=1, sr_seed=seed + 102)
+
+
+def check_2d_tiles(q2, x, tiles):
+    """2D outputs on sampled 16-row tile rows against the oracle: row codes,
+    plain tile scales, the W^T codes of those tiles' columns (the same codes
+    transposed, the pages' "row- and column-wise quantization agree"), and
+    both MMA scale layouts at the positions those tiles fill."""
+    R, C = x.shape
+    sg = O.global_scale(O.amax(x))
+    assert np.float32(q2.global_scale.item()) == np.float32(sg)
+    got = O.quantize_2d_tiles(x, sg, tiles)
+    codes = q2.codes.cpu().numpy()
+    scales = q2.scales.cpu().numpy() if q2.scales is not None else None
+    ccol = q2.codes_col.cpu().numpy() if q2.codes_col is not None else None
+    mrow = q2.scales_mma.cpu().numpy() if q2.scales_mma is not None else None
+    mcol = q2.scales_mma_col.cpu().numpy() if q2.scales_mma_col is not None else None
+    kb_row, kb_col = C // 16, R // 16
+    for tr in tiles:
+        oc, osc = got[tr]
+        assert np.array_equal(codes[16 * tr:16 * tr + 16], oc), f"row codes, tile row {tr}"
+        if scales is not None:
+            assert np.array_equal(scales[tr], osc), f"tile scales, tile row {tr}"
+        if ccol is not None:
+            nib = unpack_codes(oc)                          # [16 x C] codes of rows 16tr .. 16tr+15
+            exp = nib.T                                     # [C x 16]: W^T rows, K positions 16tr ..
+            exp_bytes = (exp[:, 0::2] | (exp[:, 1::2] << 4)).astype(np.uint8)
+            assert np.array_equal(ccol[:, 8 * tr:8 * tr + 8], exp_bytes), f"W^T codes, tile row {tr}"
+        if mrow is not None:
+            ck = (kb_row + 3) // 4
+            r = np.arange(16 * tr, 16 * tr + 16)[:, None]
+            b = np.arange(kb_row)[None, :]
+            off = ((r // 128) * ck + b // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + (b % 4)
+            assert np.array_equal(mrow[off], np.broadcast_to(osc, (16, kb_row))), f"MMA scales, tile row {tr}"
+        if mcol is not None:
+            ck = (kb_col + 3) // 4
+            c = np.arange(C)
+            off = ((c // 128) * ck + tr // 4) * 512 + (c % 32) * 16 + ((c // 32) % 4) * 4 + (tr % 4)
+            assert np.array_equal(mcol[off], osc[c // 16]), f"MMA scales of W^T, tile row {tr}"
+    return sg
 
 
 def test_quantizer_max_size_rowwise():
@@ -146,6 +185,82 @@ def test_quantizer_max_size_rowwise():
     q = N.quantize_1d(to_device_bf16(x), plain_scales=False)
     torch.cuda.synchronize()
     check_quantized_rows(q, x, sample_rows(x.shape[0], 6, seed=9))
+
+
+@pytest.mark.parametrize("dist", ["outliers"])
+def test_quantizer_max_size_all_modes(dist):
+    """2^30 elements (262144 x 4096 bf16, a 2 GiB input: byte offsets past
+    2^31) through the 2D quantizer (row codes, W^T codes, plain and both MMA
+    scale layouts), the row-wise RHT + SR quantizer and the transposed RHT +
+    SR quantizer, each on sampled rows / tile rows against the oracle, which
+    computes the tensor amax over the whole (rotated) tensor."""
+    n = 1 << 30
+    seed = G.seeds("sweep")[0] + 998
+    x = G.sweep_tensor(n, dist, seed)
+    R, C = x.shape
+    xd = to_device_bf16(x)
+    rows = sample_rows(R, 5, seed=10)
+    q2 = N.quantize_2d(xd, columnwise=True)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error() == 0
+    check_2d_tiles(q2, x, sorted(set(r // 16 for r in rows)))
+    del q2
+    torch.cuda.empty_cache()
+    q3 = N.quantize_1d(xd, rht=True, rht_seed=seed + 100, rounding=N.NVFP4_SR, sr_seed=seed + 101,
+                       plain_scales=False)
+    torch.cuda.synchronize()
+    check_quantized_rows(q3, x, rows, rht=True, rht_seed=seed + 100, rounding=1, sr_seed=seed + 101)
+    del q3
+    torch.cuda.empty_cache()
+    q4 = N.quantize_1d(xd, transpose=True, rht=True, rht_seed=seed + 100, rounding=N.NVFP4_SR, sr_seed=seed + 102,
+                       plain_scales=False)
+    torch.cuda.synchronize()
+    check_quantized_rows(q4, x, sample_rows(C, 5, seed=11), transpose=True, rht=True, rht_seed=seed + 100,
+                         rounding=1, sr_seed=seed + 102)
+
+
+@pytest.mark.parametrize("mode", [N.NVFP4_SCALE_1D, N.NVFP4_SCALE_2D])
+@pytest.mark.parametrize("out_dtype", [N.NVFP4_OUT_F32, N.NVFP4_OUT_BF16])
+def test_dequantize_full_size(mode, out_dtype):
+    """Dequantize at the step's activation size (16384 x 8192): the GPU's
+    codes are first checked against the oracle on sampled rows, then the GPU
+    dequantization of those rows against the oracle's dequantization of its
+    own codes (bf16 output: the binary32 value rounded to nearest even)."""
+    t, h = G.MLP_STEP["tokens"], G.MLP_STEP["hidden"]
+    seed = G.seeds("mlp_step")[0] + 30 + mode
+    x = G.activation(t, h, seed) if mode == N.NVFP4_SCALE_1D else G.weight(t, h, seed)
+    xd = to_device_bf16(x)
+    rows = sample_rows(t, 6, seed=12)
+    if mode == N.NVFP4_SCALE_1D:
+        q = N.quantize_1d(xd, mma_scales=False)
+        torch.cuda.synchronize()
+        sg = O.global_scale(O.amax(x))
+        got = O.quantize_1d_rows(x, sg, rows)
+        codes, scales = q.codes.cpu().numpy(), q.scales.cpu().numpy()
+        exp = {}
+        for r in rows:
+            assert np.array_equal(codes[r], got[r][0]) and np.array_equal(scales[r], got[r][1])
+            exp[r] = O.dequantize(got[r][0][None], got[r][1][None], 0, sg, 1, h)[0]
+    else:
+        q = N.quantize_2d(xd, columnwise=False, mma_scales=False)
+        torch.cuda.synchronize()
+        tiles = sorted(set(r // 16 for r in rows))
+        sg = check_2d_tiles(q, x, tiles)
+        got = O.quantize_2d_tiles(x, sg, tiles)
+        exp = {}
+        for r in rows:
+            oc, osc = got[r // 16]
+            exp[r] = O.dequantize(oc, osc[None], 1, sg, 16, h)[r % 16]
+    out = N.dequantize(q, scale_mode=mode, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error() == 0
+    for r in rows:
+        g = out[r].cpu()
+        if out_dtype == N.NVFP4_OUT_F32:
+            assert np.array_equal(g.numpy().view(np.uint32), exp[r].view(np.uint32)), f"row {r}"
+        else:
+            ref = torch.from_numpy(exp[r]).to(torch.bfloat16)
+            assert torch.equal(g.view(torch.int16), ref.view(torch.int16)), f"row {r}"
 
 
 def test_mlp_step_full_size():

@@ -130,3 +130,42 @@ def test_gemm_wgrad_rotation_cancels():
     scale = np.abs(G.bf16_bits_to_f32(dy)).astype(np.float64).T @ np.abs(G.bf16_bits_to_f32(x)).astype(np.float64)
     assert np.abs(cg - exact).max() <= 0.25 * scale.max()
     assert np.corrcoef(cg.ravel(), exact.ravel())[0, 1] > 0.9
+
+
+@pytest.mark.parametrize("mags", [(1e-18, 1e-18), (1e-25, 1e-12), (1e-30, 1e-30)])
+@pytest.mark.parametrize("out_dtype", [N.NVFP4_OUT_F32, N.NVFP4_OUT_BF16])
+def test_gemm_extreme_global_scales(mags, out_dtype):
+    """Operands whose global scales are so small that their product
+    alpha = RN(s_gA * s_gB) is not a normal binary32 number: amax 1e-18 on
+    both sides gives s_g near 3.7e-22 and alpha near 1.4e-43 (subnormal,
+    about 7 significant bits).  C itself is a normal number, and must meet the
+    2e-3 * sum|a b| bound against the float64 product of the dequantized
+    operands.  At 1e-30 C lies below the binary32 range: there the bound gets
+    the format's own floor, half its smallest subnormal (2^-150; bf16 shares
+    the exponent range, half its smallest subnormal is 2^-134)."""
+    M, Nn, K = 136, 264, 256
+    ma, mb = mags
+    a_bits = G.make_tensor(M, K, seed=91, dist="normal", scale=ma)
+    b_bits = G.make_tensor(Nn, K, seed=92, dist="normal", scale=mb)
+    a, b, a_hat, b_hat = quantized_pair(a_bits, b_bits)
+    sa, sb = float(a.global_scale.item()), float(b.global_scale.item())
+    prod = np.float32(sa) * np.float32(sb)
+    assert prod < np.float32(2.0 ** -126)          # alpha would be subnormal or zero
+    c = N.gemm(a.codes, a.scales_mma, a.global_scale, b.codes, b.scales_mma, b.global_scale, M, Nn, K,
+               out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error() == 0
+    cg = c.float().cpu().numpy().astype(np.float64)
+    ref, s = O.gemm_reference(a_hat, b_hat)
+    err = np.abs(cg - ref)
+    bf16 = out_dtype == N.NVFP4_OUT_BF16
+    if bf16:
+        err = np.maximum(err - bf16_half_ulp(ref), 0.0)
+    floor = 2.0 ** -134 if bf16 else 2.0 ** -150
+    assert np.isfinite(cg).all()
+    bad = err > TOL * s + floor
+    assert not bad.any(), f"{bad.sum()} out of tolerance; worst {(err / np.maximum(s, 1e-300)).max()}"
+    if ma == mb == 1e-30:
+        assert (np.abs(ref) < 2.0 ** -149).all()     # the case really is below the binary32 range
+    else:
+        assert (np.abs(ref[np.abs(ref) > 0]) >= 2.0 ** -126).mean() > 0.99
