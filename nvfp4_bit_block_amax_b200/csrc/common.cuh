@@ -125,6 +125,47 @@ inline PhiloxKeys philox_round_keys(uint64_t key) {
     }
     return r;
 }
+// The same generator on the host: word 0 of Philox4x32-10 at counter
+// (0, 0, 1, 0) under key `key` -- the RHT sign word (bit j set <=> d_j = -1).
+inline uint32_t rht_sign_word_host(uint64_t key) {
+    const PhiloxKeys k = philox_round_keys(key);
+    uint32_t c0 = 0u, c1 = 0u, c2 = 1u, c3 = 0u;
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k.k[2 * r];
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k.k[2 * r + 1];
+        c1 = (uint32_t)p1;
+        c3 = (uint32_t)p0;
+        c0 = n0;
+        c2 = n2;
+    }
+    return c0;
+}
+
+// Sign of each of the 16 positions of a chunk as a word to fold into the
+// bf16 -> binary32 unpack: 0x80000000 where d_j = -1, else 0.
+struct SignWords {
+    uint32_t m[16];
+};
+inline SignWords rht_sign_words_host(uint64_t rht_seed) {
+    const uint32_t d = rht_sign_word_host(rht_seed) & 0xFFFFu;
+    SignWords s;
+    for (int j = 0; j < 16; ++j) s.m[j] = ((d >> j) & 1u) ? 0x80000000u : 0u;
+    return s;
+}
+// bf16 halves of a packed word -> binary32 with a sign word applied: the low
+// half as w * 2^16 + m (adding 2^31 flips the sign bit, nothing else), the
+// high half as (w & 0xFFFF0000) ^ m -- one instruction each.
+__device__ __forceinline__ float bf16_lo_signed(uint32_t w, uint32_t m) {
+    uint32_t d;
+    asm("mad.lo.u32 %0, %1, 65536, %2;" : "=r"(d) : "r"(w), "r"(m));
+    return __uint_as_float(d);
+}
+__device__ __forceinline__ float bf16_hi_signed(uint32_t w, uint32_t m) {
+    return __uint_as_float((w & 0xFFFF0000u) ^ m);
+}
+
 __device__ __forceinline__ uint4 philox4x32_10_keys(uint4 c, const PhiloxKeys& keys) {
 #pragma unroll
     for (int r = 0; r < 10; ++r) {

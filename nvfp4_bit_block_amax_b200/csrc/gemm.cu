@@ -691,6 +691,12 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 // its scales are in TMEM (which implies its stage has landed) and when its
 // epilogue has drained the accumulator.  Per SM this moves 38 KB per 64 K
 // columns instead of 54 KB: the single-SM tile is L2-bandwidth bound.
+// Per CTA 14 warps: warp 0 the TMA producer, warp 1 the MMA issuer (CTA 0),
+// warps 2..5 copy block scales to tensor memory and nothing else (one per
+// TMEM lane quarter), warps 6..13 the epilogue (two per lane quarter, one
+// per 128-column half).  Keeping the scale copies off the epilogue warps
+// means the scales of the next stages are in place while a finished tile is
+// drained and stored.
 constexpr int P_STAGES = 5;
 static_assert(SF_COL + P_STAGES * 48 <= TMEM_COLS, "scale buffers must fit in tensor memory");
 constexpr int P_A_STAGE = 128 * BKB;                 // 16 KB
@@ -703,6 +709,7 @@ constexpr int P_OFF_BAR = P_OFF_SFB + P_STAGES * SFB_STAGE;
 constexpr int P_NUM_BARS = 3 * P_STAGES + 3;   // full, empty, sf_full per stage; tmem_full/empty, drain
 constexpr int P_OFF_MISC = P_OFF_BAR + P_NUM_BARS * 8;
 constexpr int P_SMEM_BYTES = P_OFF_MISC + 16 + 1024;
+constexpr int P_NUM_THREADS = 448;                  // 14 warps: producer, MMA, 4 scale warps, 8 epilogue warps
 // M = 256 (pair), N = 256, E2M1 x E2M1, UE4M3 scales, K-major.
 constexpr uint32_t kIdescPair = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 
@@ -797,7 +804,7 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
 }
 
 template <bool MX>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(P_NUM_THREADS, 1)
 gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, KParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -921,38 +928,18 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
             while (!mbar_try_cluster(bar_drain, 0) && globaltimer() - t0 < kWaitLimitNs) {}
         }
     } else if (warp < 6) {
-        // ------------------------------- scales -> TMEM, and the epilogue ----
+        // -------------------------------------------------- scales -> TMEM ----
+        // Warp q of this group owns TMEM lanes 32q..32q+31 (q = warp % 4) and
+        // does nothing else, so the block scales of the next stages are in
+        // tensor memory while the epilogue warps drain and store.
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float2 alpha = out_scales(p);
         int s = 0;
-        uint32_t phase = 0, acc_phase = 0;
+        uint32_t phase = 0;
         bool ok = true;
-        int prev_tile = -1;
-        uint32_t amax_acc = 0;   // max |C| of this thread's drained rows (binary32 bits)
         for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
             for (int kb = 0; kb < k_blocks; ++kb) {
-                // As in the single-SM kernel: wait for the stage, draining the
-                // previous tile's accumulator half the moment it is complete.
-                {
-                    const unsigned long long t0 = globaltimer();
-                    while (true) {
-                        if (prev_tile >= 0 && mbar_test_cluster(bar_tfull, acc_phase)) {
-                            if (!epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty,
-                                                    acc_phase, abort_flag, amax_acc)) { ok = false; break; }
-                            prev_tile = -1;
-                        }
-                        if (mbar_test_cluster(bar_full + 8 * s, phase)) break;
-                        if (*abort_flag) { ok = false; break; }
-                        if (globaltimer() - t0 > kWaitLimitNs) {
-                            *abort_flag = 1;
-                            atomicExch(&g_error_word, 1u);
-                            ok = false;
-                            break;
-                        }
-                    }
-                    if (!ok) break;
-                }
+                if (!mbar_wait(bar_full + 8 * s, phase, abort_flag)) { ok = false; break; }
                 const uint32_t sfa_s = sbase + P_OFF_SFA + s * SFA_STAGE + 16 * lane;
                 const uint32_t sfb_s = sbase + P_OFF_SFB + s * SFB_STAGE + 16 * lane;
                 uint32_t ra[16], rb0[16], rb1[16];
@@ -984,26 +971,17 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
                 }
                 if (++s == P_STAGES) { s = 0; phase ^= 1; }
             }
-            if (ok && prev_tile >= 0) {
-                if (!epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase,
-                                        abort_flag, amax_acc)) ok = false;
-                prev_tile = -1;
-            }
-            if (ok) prev_tile = tile;
         }
-        if (ok && prev_tile >= 0)
-            epilogue_half_pair(p, prev_tile, 0, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase, abort_flag,
-                               amax_acc);
-        __syncwarp();
-        if (p.c_amax) amax_publish(p.c_amax, amax_acc);
     } else {
-        // ---------------------------------------- epilogue, columns 128..255 ----
-        const int q = warp & 3;
+        // ----------------------------------------------------------- epilogue ----
+        // warps 6..9: columns 0..127, warps 10..13: columns 128..255, of the
+        // TMEM lane quarter warp % 4
+        const int q = warp & 3, half = (warp - 6) >> 2;
         const float2 alpha = out_scales(p);
         uint32_t acc_phase = 0;
         uint32_t amax_acc = 0;
         for (int tile = cluster; tile < num_tiles; tile += n_clusters)
-            if (!epilogue_half_pair(p, tile, 1, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase,
+            if (!epilogue_half_pair(p, tile, half, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase,
                                     abort_flag, amax_acc)) break;
         __syncwarp();
         if (p.c_amax) amax_publish(p.c_amax, amax_acc);
@@ -1088,7 +1066,7 @@ DeviceInfo device_info() {
         }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(2 * (n / 2));
-        cfg.blockDim = dim3(NUM_THREADS);
+        cfg.blockDim = dim3(P_NUM_THREADS);
         cfg.dynamicSmemBytes = P_SMEM_BYTES;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1163,7 +1141,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     const int clusters = tiles < dev.pair_clusters ? tiles : dev.pair_clusters;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * clusters);
-    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.blockDim = dim3(P_NUM_THREADS);
     cfg.dynamicSmemBytes = P_SMEM_BYTES;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];

@@ -109,6 +109,7 @@ struct Params {
     int64_t rows, cols, ld;
     uint64_t rht_seed, sr_seed;
     PhiloxKeys sr_keys;           // round keys of sr_seed
+    SignWords rht_sign;           // RHT signs of the 16 positions of a chunk, as unpack masks
     uint8_t* codes;
     uint8_t* scales;
     uint8_t* scales_mma;
@@ -356,6 +357,109 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
         }
     }
     if (AMAX_ONLY) write_partial(amax_bits, p.partials);
+}
+
+// ------------------------------------- rowwise 1D, stochastic rounding ------
+// Stochastic rounding needs 16 Philox bits per element, which makes the
+// encode pass instruction-bound: this kernel keeps the per-block bookkeeping
+// small by giving each thread 64 consecutive elements of a Q row (4 blocks,
+// one 128-byte span): one Philox counter base, one 32-byte code store pair,
+// and the 4 block scales of a row are exactly one 32-bit word of the GEMM
+// scale layout.  A warp takes 32 such units (2048 columns) of one row at a
+// time; segments are dealt to the warps in order.  RHT (16-point): the signs
+// are folded into the bf16 unpack (sign words from the parameter bank).
+template <bool RHT>
+__global__ void __launch_bounds__(kThreads) rows_sr_kernel(Params p) {
+    __shared__ float s_rtab[128];
+    float sg, t;
+    global_scales(p, sg, t);
+    const ScaleCtx ctx = make_scale_ctx(sg, t, s_rtab);
+    const int lane = threadIdx.x & 31;
+    const int64_t C = p.cols;
+    const int64_t upr = (C + 63) >> 6;                   // 64-element units per row
+    const int64_t spr = (upr + 31) >> 5;                 // 32-unit warp segments per row
+    const int64_t items = p.rows * spr;
+    const int64_t nwarps = (int64_t)gridDim.x * (kThreads / 32);
+    int64_t item = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+    if (item >= items) return;                           // (no block-wide barrier below)
+    int64_t row = item / spr, seg = item - row * spr;
+    const int64_t step_rows = nwarps / spr, step_seg = nwarps - step_rows * spr;
+    const bool a32 = ((reinterpret_cast<uintptr_t>(p.x) & 31u) == 0) && ((p.ld & 15) == 0);
+    const bool c16 = ((C & 63) == 0) && ((reinterpret_cast<uintptr_t>(p.codes) & 15u) == 0);
+    for (; item < items; item += nwarps) {
+        const int64_t col0 = ((seg << 5) + lane) << 6;
+        const int nb = col0 < C ? (int)min((int64_t)4, (C - col0) >> 4) : 0;   // blocks of this unit inside the row
+        uint32_t w[4][8];
+        const uint16_t* src = p.x + row * p.ld + col0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            if (b < nb) load_block(src + 16 * b, a32, w[b]);
+            else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) w[b][j] = 0u;
+            }
+        }
+        const uint64_t g0 = (uint64_t)(row * C + col0) >> 3;   // Philox counter of the unit's first 8 elements
+        uint32_t cw[8];
+        uint32_t sword = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            float y[16];
+            float bmax;
+            if (RHT) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    y[2 * j] = bf16_lo_signed(w[b][j], p.rht_sign.m[2 * j]);
+                    y[2 * j + 1] = bf16_hi_signed(w[b][j], p.rht_sign.m[2 * j + 1]);
+                }
+                rht16_butterflies(y);
+                scale_regs(y, 0.25f);
+                bmax = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) bmax = max3f(bmax, fabsf(y[j]), fabsf(y[j + 1]));
+            } else {
+                uint32_t acc = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc = absmax2(acc, w[b][j]);
+                bmax = __uint_as_float(absmax2_fold(acc));
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    y[2 * j] = bf16_lo(w[b][j]);
+                    y[2 * j + 1] = bf16_hi(w[b][j]);
+                }
+            }
+            // blocks past the row's end hold zeros: zero scale, codes not stored
+            const BlockScale bs = block_scale(bmax, ctx);
+            encode16<true>(y, bs, p.sr_keys, g0 + 2 * b, cw[2 * b], cw[2 * b + 1]);
+            if (b < nb) sword |= bs.code << (8 * b);
+        }
+        if (nb > 0) {
+            uint8_t* cp = p.codes + row * (C >> 1) + (col0 >> 1);
+            if (nb == 4 && c16) {
+                *reinterpret_cast<uint4*>(cp) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                *reinterpret_cast<uint4*>(cp + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+            } else {
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    if (b < nb) *reinterpret_cast<uint2*>(cp + 8 * b) = make_uint2(cw[2 * b], cw[2 * b + 1]);
+            }
+            if (p.scales) {
+                uint8_t* sp = p.scales + row * (C >> 4) + (col0 >> 4);
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    if (b < nb) sp[b] = (uint8_t)(sword >> (8 * b));
+            }
+            // blocks 4g .. 4g+3 of the row: one word of the GEMM layout (zeros past the row's end)
+            if (p.scales_mma)
+                *reinterpret_cast<uint32_t*>(p.scales_mma + mma_scale_offset(row, col0 >> 4, p.chunks_k)) = sword;
+        }
+        row += step_rows;
+        seg += step_seg;
+        if (seg >= spr) {
+            seg -= spr;
+            ++row;
+        }
+    }
 }
 
 // ---------------------------------------------- transposed 1D (Q = x^T) -------
@@ -767,6 +871,14 @@ int launch_amax_plain(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
     return g;
 }
 
+// Grid of the SR row-wise encode pass: every resident CTA of the device,
+// no more than there are warp segments to hand out.
+template <bool RHT>
+int rows_sr_grid(const Params& p) {
+    const int64_t segs = p.rows * ((((p.cols + 63) >> 6) + 31) >> 5);
+    return grid_for(rows_sr_kernel<RHT>, (segs + 7) / 8);
+}
+
 template <bool RHT, bool SR, int LOGM = 0>
 cudaError_t run_rows(Params p, const float* given, cudaStream_t s, int* launches) {
     const int64_t units = p.rows * ((p.cols + 511) >> 9);
@@ -782,7 +894,8 @@ cudaError_t run_rows(Params p, const float* given, cudaStream_t s, int* launches
     } else {
         p.n_partials = launch_amax_plain(p.x, p.rows, p.cols, p.ld, p.partials, s);
     }
-    rows_kernel<RHT, SR, false, LOGM><<<g, kThreads, 0, s>>>(p);
+    if (SR && LOGM == 0) rows_sr_kernel<RHT><<<rows_sr_grid<RHT>(p), kThreads, 0, s>>>(p);
+    else rows_kernel<RHT, SR, false, LOGM><<<g, kThreads, 0, s>>>(p);
     *launches += 2;
     return cudaGetLastError();
 }
@@ -827,6 +940,7 @@ cudaError_t launch_quantize_1d(const QuantArgs& a, cudaStream_t s, int* launches
     p.rht_seed = a.rht_seed;
     p.sr_seed = a.sr_seed;
     p.sr_keys = philox_round_keys(a.sr_seed);
+    p.rht_sign = rht_sign_words_host(a.rht_seed);
     p.codes = a.codes;
     p.scales = a.scales;
     p.scales_mma = a.scales_mma;
@@ -905,7 +1019,7 @@ cudaError_t launch_quantize_dual(const QuantArgs& r, const QuantArgs& t, cudaStr
     pt.partials2 = nullptr;
     const int64_t units = r.rows * ((r.cols + 511) >> 9);
     const int64_t wneed = (units + 1) / 2;
-    if (sr_r) rows_kernel<false, true, false><<<grid_for(rows_kernel<false, true, false>, (wneed + 7) / 8), kThreads, 0, s>>>(pr);
+    if (sr_r) rows_sr_kernel<false><<<rows_sr_grid<false>(pr), kThreads, 0, s>>>(pr);
     else rows_kernel<false, false, false><<<grid_for(rows_kernel<false, false, false>, (wneed + 7) / 8), kThreads, 0, s>>>(pr);
     if (sr_t) cols_kernel<true, true, false><<<gc, kThreads, 0, s>>>(pt);
     else cols_kernel<true, false, false><<<gc, kThreads, 0, s>>>(pt);
