@@ -696,7 +696,10 @@ gemm_nvf4_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 // TMEM lane quarter), warps 6..13 the epilogue (two per lane quarter, one
 // per 128-column half).  Keeping the scale copies off the epilogue warps
 // means the scales of the next stages are in place while a finished tile is
-// drained and stored.
+// drained and stored.  The epilogue stores C through the TMA: each warp
+// stages 32 rows x 64 bytes in shared memory and issues one bulk tensor
+// store per chunk, so C is written in whole lines and the hardware drops the
+// rows and columns past the edges of a ragged tile.
 constexpr int P_STAGES = 5;
 static_assert(SF_COL + P_STAGES * 48 <= TMEM_COLS, "scale buffers must fit in tensor memory");
 constexpr int P_A_STAGE = 128 * BKB;                 // 16 KB
@@ -708,14 +711,53 @@ constexpr int P_OFF_SFB = P_OFF_SFA + P_STAGES * SFA_STAGE;
 constexpr int P_OFF_BAR = P_OFF_SFB + P_STAGES * SFB_STAGE;
 constexpr int P_NUM_BARS = 3 * P_STAGES + 3;   // full, empty, sf_full per stage; tmem_full/empty, drain
 constexpr int P_OFF_MISC = P_OFF_BAR + P_NUM_BARS * 8;
-constexpr int P_SMEM_BYTES = P_OFF_MISC + 16 + 1024;
+constexpr int P_OFF_EPI = (P_OFF_MISC + 16 + 1023) / 1024 * 1024;   // output staging, one 2 KB buffer per epilogue warp
+constexpr int EPI_BUF = 2048;                                      // 32 rows x 64 bytes, 64-byte swizzle
+constexpr int P_SMEM_BYTES = P_OFF_EPI + 8 * EPI_BUF + 1024;
 constexpr int P_NUM_THREADS = 448;                  // 14 warps: producer, MMA, 4 scale warps, 8 epilogue warps
 // M = 256 (pair), N = 256, E2M1 x E2M1, UE4M3 scales, K-major.
 constexpr uint32_t kIdescPair = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 
+// Output store through the tensor-memory-access unit: a 32-row x 64-byte
+// chunk staged in shared memory (64-byte swizzle: 16-byte unit u of row r
+// sits at unit u ^ ((r >> 1) & 3)) is written to C by one bulk tensor store;
+// rows and columns past the tensor's edge are dropped by the hardware.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// Stage one 32-row x 64-byte chunk (this lane's row: 16 words) and store it.
+__device__ __forceinline__ void store_chunk(const CUtensorMap* map_c, uint32_t buf, int lane, const uint32_t* w, int col,
+                                            int row0, bool first) {
+    if (!first) {
+        if (lane == 0) bulk_wait_read0();   // the buffer's previous chunk has been read out
+        __syncwarp();
+    }
+    const uint32_t rowaddr = buf + lane * 64;
+    const uint32_t sw = (lane >> 1) & 3;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) sts128(rowaddr + ((u ^ sw) << 4), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(map_c, buf, col, row0);
+        bulk_commit();
+    }
+}
+
 __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, int half, int q, int lane, uint32_t rank,
                                                    uint32_t tmem, float2 alpha, uint32_t bar_tfull, uint32_t bar_tempty,
-                                                   uint32_t& acc_phase, volatile int* abort_flag, uint32_t& amax_acc) {
+                                                   uint32_t& acc_phase, volatile int* abort_flag, uint32_t& amax_acc,
+                                                   const CUtensorMap* map_c, uint32_t buf, bool& first) {
     if (!mbar_wait_cluster(bar_tfull, acc_phase, abort_flag)) return false;
     tc_fence_after();
     int tm, tn;
@@ -753,59 +795,53 @@ __device__ __forceinline__ bool epilogue_half_pair(const KParams& p, int tile, i
         }
         release();
         if (p.c_amax) amax_acc = max(amax_acc, packed_row_amax(packed, ncols, row < p.M));
-        if (row < p.M && ncols > 0) {
-            __nv_bfloat16* crow = reinterpret_cast<__nv_bfloat16*>(p.c) + (int64_t)row * p.ldc + col0;
-            if (ncols >= 128) {
+        const int row0 = tm * 256 + (int)rank * 128 + q * 32;
+        if (row0 < p.M && ncols > 0) {
 #pragma unroll
-                for (int g = 0; g < 16; ++g)
-                    *reinterpret_cast<uint4*>(crow + 8 * g) =
-                        make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
-            } else {
-#pragma unroll
-                for (int g = 0; g < 64; ++g) {
-                    if (2 * g + 1 < ncols) reinterpret_cast<uint32_t*>(crow)[g] = packed[g];
-                    else if (2 * g < ncols) reinterpret_cast<uint16_t*>(crow)[2 * g] = (uint16_t)(packed[g] & 0xFFFFu);
-                }
+            for (int k = 0; k < 4; ++k) {
+                if (32 * k < ncols) store_chunk(map_c, buf, lane, packed + 16 * k, col0 + 32 * k, row0, first);
+                first = false;
             }
         }
     } else {
-        float* crow = reinterpret_cast<float*>(p.c) + (int64_t)row * p.ldc + col0;
+        // fp32: 8 chunks of 16 columns (64 bytes per row), two chunks per TMEM load of 32 columns
+        const int row0 = tm * 256 + (int)rank * 128 + q * 32;
+        const bool live = row0 < p.M && ncols > 0;
         float fmax = 0.0f;
 #pragma unroll 1
         for (int i = 0; i < 4; ++i) {
             uint32_t v[32];
             tc_ld_32x32b_x32(taddr + 32 * i, v);
             tc_wait_ld();
-            if (row < p.M) {
+            if (i == 3) release();
+            uint32_t f[32];
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const int cc = 32 * i + 4 * g;
-                    const float2 f01 = scale_out2(v[4 * g], v[4 * g + 1], alpha);
-                    const float2 f23 = scale_out2(v[4 * g + 2], v[4 * g + 3], alpha);
-                    const float4 f = make_float4(f01.x, f01.y, f23.x, f23.y);
-                    if (cc + 4 <= ncols) {
-                        *reinterpret_cast<float4*>(crow + cc) = f;
-                        fmax = fmaxf(fmaxf(fmaxf(fmax, fabsf(f.x)), fmaxf(fabsf(f.y), fabsf(f.z))), fabsf(f.w));
-                    } else {
-                        const float ff[4] = {f.x, f.y, f.z, f.w};
-                        for (int e = 0; e < 4; ++e)
-                            if (cc + e < ncols) {
-                                crow[cc + e] = ff[e];
-                                fmax = fmaxf(fmax, fabsf(ff[e]));
-                            }
-                    }
+            for (int g = 0; g < 16; ++g) {
+                const float2 o = scale_out2(v[2 * g], v[2 * g + 1], alpha);
+                f[2 * g] = __float_as_uint(o.x);
+                f[2 * g + 1] = __float_as_uint(o.y);
+                if (row < p.M) {
+                    if (32 * i + 2 * g < ncols) fmax = fmaxf(fmax, fabsf(o.x));
+                    if (32 * i + 2 * g + 1 < ncols) fmax = fmaxf(fmax, fabsf(o.y));
+                }
+            }
+            if (live) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (32 * i + 16 * h < ncols) store_chunk(map_c, buf, lane, f + 16 * h, col0 + 32 * i + 16 * h, row0, first);
+                    first = false;
                 }
             }
         }
         amax_acc = max(amax_acc, __float_as_uint(fmax));
-        release();
     }
     return true;
 }
 
 template <bool MX>
 __global__ void __launch_bounds__(P_NUM_THREADS, 1)
-gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, KParams p) {
+gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                      const __grid_constant__ CUtensorMap map_c, KParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -978,11 +1014,14 @@ gemm_nvf4_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_co
         // TMEM lane quarter warp % 4
         const int q = warp & 3, half = (warp - 6) >> 2;
         const float2 alpha = out_scales(p);
+        const uint32_t buf = sbase + P_OFF_EPI + (warp - 6) * EPI_BUF;
         uint32_t acc_phase = 0;
         uint32_t amax_acc = 0;
+        bool first = true;
         for (int tile = cluster; tile < num_tiles; tile += n_clusters)
             if (!epilogue_half_pair(p, tile, half, q, lane, rank, tmem, alpha, bar_tfull, bar_tempty, acc_phase,
-                                    abort_flag, amax_acc)) break;
+                                    abort_flag, amax_acc, &map_c, buf, first)) break;
+        if (lane == 0) bulk_wait0();    // every store of this warp has completed
         __syncwarp();
         if (p.c_amax) amax_publish(p.c_amax, amax_acc);
     }
@@ -1039,6 +1078,19 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t k,
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ldc, bool bf16) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const int esz = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ldc * esz)};
+    cuuint32_t box[2] = {(cuuint32_t)(64 / esz), 32};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1132,8 +1184,9 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
         return cudaGetLastError();
     }
     // CTA pairs: 256 x 256 tiles, each CTA loads 128-row boxes of A and B
-    CUtensorMap ma, mb;
-    if (!make_code_map(&ma, g.a, g.M, g.K, 128) || !make_code_map(&mb, g.b, g.N, g.K, 128))
+    CUtensorMap ma, mb, mc;
+    if (!make_code_map(&ma, g.a, g.M, g.K, 128) || !make_code_map(&mb, g.b, g.N, g.K, 128) ||
+        !make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.out_bf16 != 0))
         return cudaErrorInvalidValue;
     p.tiles_m = (int)ceil_div(g.M, 256);
     p.group_m = group_for(256, g.K, p.tiles_m);
@@ -1151,8 +1204,8 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return p.mx ? cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<true>, ma, mb, p)
-                : cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<false>, ma, mb, p);
+    return p.mx ? cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<true>, ma, mb, mc, p)
+                : cudaLaunchKernelEx(&cfg, gemm_nvf4_pair_kernel<false>, ma, mb, mc, p);
 }
 
 unsigned int read_and_clear_error_word(cudaStream_t s, cudaError_t* err) {
