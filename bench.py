@@ -55,7 +55,7 @@ def parse():
                     choices=["gemm", "gemm_amax", "quantize_1d", "quantize_1d_sr", "quantize_2d", "rht_t_sr",
                              "rht_t_rne", "quantize_1d_from_amax", "quantize_2d_from_amax", "mx_quantize",
                              "mx_gemm", "quantize_dual", "quantize_dual_sr",
-                             "dequantize", "rht_sr", "rht_rne"],
+                             "dequantize", "rht_sr", "rht_rne", "mx_dequantize", "scales_to_mma"],
                     help="time one kernel family alone on --shape (profiling mode)")
     ap.add_argument("--shape", default=None, help="M,N,K for gemm; rows,cols otherwise")
     ap.add_argument("--sweep", action="store_true",
@@ -832,6 +832,15 @@ def micro(args):
             sm2 = torch.empty(N.nvfp4_mma_scale_bytes(C, R), dtype=torch.uint8, device=dev)
             fn = lambda: N.nvfp4_quantize_2d(x, R, C, C, codes, cc, None, smma, sm2, gs, ws, ws.numel(), s)
             work = R * C * (2 + 0.5 + 0.5 + 2 / 16)
+        elif args.op == "mx_dequantize":
+            sc = torch.randint(118, 136, (R, C // 32), dtype=torch.uint8, device=dev, generator=g)
+            out = torch.empty(R, C, dtype=torch.bfloat16, device=dev)
+            fn = lambda: N.nvfp4_mxfp4_dequantize(codes, sc, R, C, N.NVFP4_OUT_BF16, out, s)
+            work = R * C * (0.5 + 1 / 32 + 2)
+        elif args.op == "scales_to_mma":
+            sc = torch.randint(0x30, 0x40, (R, C // 16), dtype=torch.uint8, device=dev, generator=g)
+            fn = lambda: N.nvfp4_scales_to_mma(sc, 0, R, C, smma, s)
+            work = R * (C // 16) + N.nvfp4_mma_scale_bytes(R, C)
         elif args.op == "dequantize":
             sc = torch.randint(0x30, 0x40, (R, C // 16), dtype=torch.uint8, device=dev, generator=g)
             out = torch.empty(R, C, dtype=torch.bfloat16, device=dev)

@@ -350,8 +350,10 @@ __device__ __forceinline__ float2 scale_out2(uint32_t u0, uint32_t u1, float2 al
 }
 
 // Tile t -> (tm, tn).  Tiles are taken in groups of group_m M-tiles; inside a
-// group M runs fastest, then N.  The CTAs working at the same time then share
-// group_m A panels and a few B panels, which stay resident in L2.
+// group M runs fastest, then N, and odd groups walk N backwards.  The CTAs
+// working at the same time then share group_m A panels and a few B panels,
+// which stay resident in L2, and a group starts on the B panels its
+// predecessor used last (measured: dgrad DRAM reads 3.2 -> 2.6 GB per launch).
 __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& tm, int& tn) {
     const int per_group = p.group_m * p.tiles_n;
     const int g = t / per_group;
@@ -360,6 +362,7 @@ __device__ __forceinline__ void tile_coords(int t, const KParams& p, int& tm, in
     const int gm = min(p.group_m, p.tiles_m - first);
     tm = first + r % gm;
     tn = r / gm;
+    if (g & 1) tn = p.tiles_n - 1 - tn;   // serpentine: a group starts on the B panels the previous one ended on
 }
 
 // Epilogue of one column half (128 columns) of a finished tile for the

@@ -514,6 +514,10 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 uint32_t w = jp == 0 ? v[i].x : jp == 1 ? v[i].y : jp == 2 ? v[i].z : v[i].w;
+                if (RHT && LOGM == 0 && !AMAX_ONLY) {   // signs folded into the unpack (sign words from the parameter bank)
+                    y[i] = make_float2(bf16_lo_signed(w, p.rht_sign.m[i]), bf16_hi_signed(w, p.rht_sign.m[i]));
+                    continue;
+                }
                 if (RHT && ((dmask >> i) & 1u)) w ^= 0x80008000u;
                 y[i] = make_float2(bf16_lo(w), bf16_hi(w));
             }
@@ -982,6 +986,7 @@ cudaError_t launch_quantize_dual(const QuantArgs& r, const QuantArgs& t, cudaStr
     pt.rht_seed = t.rht_seed;
     pt.sr_seed = t.sr_seed;
     pt.sr_keys = philox_round_keys(t.sr_seed);
+    pt.rht_sign = rht_sign_words_host(t.rht_seed);
     pt.codes = t.codes;
     pt.scales = t.scales;
     pt.scales_mma = t.scales_mma;
