@@ -204,3 +204,21 @@ def test_scales_to_mma():
         dst = torch.empty(N.nvfp4_mma_scale_bytes(rows, k), dtype=torch.uint8, device="cuda")
         N.nvfp4_scales_to_mma(torch.from_numpy(plain).cuda(), mode, rows, k, dst)
         assert np.array_equal(dst.cpu().numpy(), mma_layout(plain, rows, k // 16, expand_2d=bool(mode)))
+
+
+@pytest.mark.parametrize("ld", [72, 96])
+@pytest.mark.parametrize("rht", [False, True])
+def test_strided_input_sr(ld, rht):
+    """Stochastic rounding (and the 16-point RHT) on a strided view: rows of
+    64 elements every `ld` elements.  ld = 72 leaves every other row 16-byte
+    but not 32-byte aligned, so the encode pass takes its two-load path."""
+    x = G.make_tensor(40, ld, seed=9 + ld, dist="laplace", scale=1e-3, outlier_frac=0.01, outlier_mode="mul",
+                      outlier_value=500.0)
+    xd = to_device_bf16(x)[:, :64]
+    q = N.quantize_1d(xd, rounding=N.NVFP4_SR, sr_seed=21, rht=rht, rht_seed=22)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error() == 0
+    oc, osc, osg = O.quantize_1d(np.ascontiguousarray(x[:, :64]), rht=rht, rht_seed=22, rounding=1, sr_seed=21)
+    assert np.array_equal(q.codes.cpu().numpy(), oc) and np.array_equal(q.scales.cpu().numpy(), osc)
+    assert np.array_equal(q.scales_mma.cpu().numpy(), mma_layout(osc, 40, 4))
+    assert q.global_scale.item() == osg
