@@ -472,9 +472,15 @@ __global__ void __launch_bounds__(kThreads) rows_sr_kernel(Params p) {
 // pieces of a chunk share a warp -- warp w: features 32w .. 32w+31; lane:
 // 16-token piece lane >> 2, 8 features from 8 * (lane & 3) -- and the
 // butterflies h >= 16 are shuffles between lanes lane ^ 4, ^ 8, ^ 16.
+// The 16-point stochastic-rounding encode stores each thread's 8-byte code
+// segments straight from registers instead (the four warps of a tile fill
+// each 32-byte sector between them): that pass is bound by instruction issue,
+// and the staging copy's shared-memory traffic and barrier cost more than the
+// narrower global stores.  With round-to-nearest the staged store is faster.
 template <bool RHT, bool SR, bool AMAX_ONLY, int LOGM = 0>
 __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
-    __shared__ __align__(16) uint8_t s_codes[AMAX_ONLY ? 16 : 256 * 64];
+    constexpr bool kDirect = RHT && SR && !AMAX_ONLY && LOGM == 0;
+    __shared__ __align__(16) uint8_t s_codes[(AMAX_ONLY || kDirect) ? 16 : 256 * 64];
     __shared__ __align__(16) uint8_t s_sc[AMAX_ONLY ? 1 : 256][8];   // [feature in tile][token block in tile]
     __shared__ float s_rtab[128];
     ScaleCtx ctx{};
@@ -594,8 +600,12 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
                 const uint32_t hi =
                     e2m1x8(q[c][8], q[c][9], q[c][10], q[c][11], q[c][12], q[c][13], q[c][14], q[c][15]);
                 const int srow = fl0 + j;
-                const int key = LOGM == 0 ? (lane & 7) : ((srow >> 3) & 7);   // = (srow >> 3) & 7
-                *reinterpret_cast<uint2*>(s_codes + srow * 64 + ((piece ^ key) * 8)) = make_uint2(lo, hi);
+                if (kDirect) {
+                    if (ok) *reinterpret_cast<uint2*>(p.codes + (f0 + j) * (T >> 1) + (t0 >> 1)) = make_uint2(lo, hi);
+                } else {
+                    const int key = LOGM == 0 ? (lane & 7) : ((srow >> 3) & 7);   // = (srow >> 3) & 7
+                    *reinterpret_cast<uint2*>(s_codes + srow * 64 + ((piece ^ key) * 8)) = make_uint2(lo, hi);
+                }
                 s_sc[srow][piece] = ok ? (uint8_t)code : (uint8_t)0;
                 if (ok && p.scales) p.scales[(f0 + j) * kb + (t0 >> 4)] = (uint8_t)code;
             }
@@ -614,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
             }
         }
         const int64_t row_bytes = min((int64_t)64, (T >> 1) - tbyte);
-        for (int k = threadIdx.x; k < 256 * 8; k += kThreads) {
+        for (int k = threadIdx.x; !kDirect && k < 256 * 8; k += kThreads) {
             const int r = k >> 3, c8 = k & 7;
             if (fbase + r < F && c8 * 8 < row_bytes) {
                 const uint2 val = *reinterpret_cast<const uint2*>(s_codes + r * 64 + ((c8 ^ ((r >> 3) & 7)) * 8));
