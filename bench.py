@@ -532,7 +532,7 @@ def e2e(torch, N, step, s, args, dist=None, world=1, dev=None):
     odw = torch.empty(step.dw.shape, dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * 2 for t in (hx, hw, hdy))
     d2h = sum(t.numel() * 2 for t in (oy, odx, odw))
-    n = max(3, min(args.steps, 10))
+    n = max(3, min(args.steps, 40))
     sets = [step, step.twin()]
     s_in, s_out = torch.cuda.Stream(device=step.dev), torch.cuda.Stream(device=step.dev)
     ev = lambda: torch.cuda.Event()

@@ -222,3 +222,23 @@ def test_strided_input_sr(ld, rht):
     assert np.array_equal(q.codes.cpu().numpy(), oc) and np.array_equal(q.scales.cpu().numpy(), osc)
     assert np.array_equal(q.scales_mma.cpu().numpy(), mma_layout(osc, 40, 4))
     assert q.global_scale.item() == osg
+
+
+@pytest.mark.parametrize("ld", [72, 264])
+@pytest.mark.parametrize("rounding", [0, 1])
+def test_strided_input_transposed_rht(ld, rounding):
+    """Q = RHT(x^T) of a strided view (tokens x 64 features every `ld`
+    elements): the transposed encode reads through the stride and writes Q's
+    rows (one per feature) whole; the SR variant stores its codes straight
+    from registers, the RNE one through shared memory."""
+    x = G.make_tensor(48, ld, seed=30 + ld, dist="laplace", scale=1e-3, outlier_frac=0.01, outlier_mode="mul",
+                      outlier_value=500.0)
+    xd = to_device_bf16(x)[:, :64]
+    q = N.quantize_1d(xd, transpose=True, rounding=rounding, sr_seed=23, rht=True, rht_seed=24)
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error() == 0
+    oc, osc, osg = O.quantize_1d(np.ascontiguousarray(x[:, :64]), transpose=True, rht=True, rht_seed=24,
+                                 rounding=rounding, sr_seed=23)
+    assert np.array_equal(q.codes.cpu().numpy(), oc) and np.array_equal(q.scales.cpu().numpy(), osc)
+    assert np.array_equal(q.scales_mma.cpu().numpy(), mma_layout(osc, 64, 3))
+    assert q.global_scale.item() == osg
