@@ -712,6 +712,17 @@ __global__ void __launch_bounds__(kThreads, 2) q2d_kernel(Params2d p) {
         uint4 v[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = ok ? ldg_stream(p.w + (r0 + i) * p.ld + c0) : make_uint4(0u, 0u, 0u, 0u);
+        // While this tile is encoded and its outputs staged (two block-wide
+        // barriers, during which no load of this CTA is in flight), pull the
+        // CTA's next tile into L2: thread r < 128 takes row r (512 bytes).
+        {
+            const int64_t nt = tile + gridDim.x;
+            if (nt < ntiles && threadIdx.x < 128) {
+                const int64_t ntr_ = nt / ntc, ntc_ = nt - ntr_ * ntc;
+                const int64_t pr = ntr_ * 128 + threadIdx.x, pc = ntc_ * 256;
+                if (pr < R) prefetch_l2(p.w + pr * p.ld + pc, (uint32_t)(min((int64_t)256, C - pc) * 2));
+            }
+        }
         uint32_t acc = 0;
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc = absmax2(absmax2(absmax2(absmax2(acc, v[i].x), v[i].y), v[i].z), v[i].w);
