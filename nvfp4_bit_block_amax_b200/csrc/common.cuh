@@ -218,6 +218,13 @@ template <int LOGM>
 __device__ __forceinline__ constexpr float rht_norm() {
     return LOGM == 0 ? 0.25f : LOGM == 1 ? 0x1.6a09e6p-3f : LOGM == 2 ? 0.125f : 0x1.6a09e6p-4f;
 }
+// The 16-point factor 1/4 commutes exactly with the maximum: every butterfly
+// value is a sum of +-bf16 values, so a multiple of 2^-133 (bf16's smallest
+// subnormal), and a quarter of it is representable in binary32 (2^-135 is a
+// multiple of binary32's subnormal step 2^-149).  So max |y / 4| = (max |y|) / 4
+// bit for bit, and an amax pass may scale its maximum once instead of every
+// element.
+constexpr float kRht16Norm = 0.25f;
 
 // Stochastic rounding onto the E2M1 grid of one scaled value v (finite):
 // between neighbours lo <= |v| < hi, f = floor(p * 2^16) with

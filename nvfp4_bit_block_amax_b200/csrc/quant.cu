@@ -312,7 +312,8 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
                     }
                     rht16_butterflies(y);
                     if (LOGM > 0) rht_cross_lanes<LOGM>(y, lane);
-                    scale_regs(y, rht_norm<LOGM>());
+                    // the 16-point amax pass applies the 1/4 to its maximum (kRht16Norm)
+                    if (!(AMAX_ONLY && LOGM == 0)) scale_regs(y, rht_norm<LOGM>());
                     bmax = 0.0f;
 #pragma unroll
                     for (int j = 0; j < 16; j += 2) bmax = max3f(bmax, fabsf(y[j]), fabsf(y[j + 1]));
@@ -356,7 +357,10 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
             }
         }
     }
-    if (AMAX_ONLY) write_partial(amax_bits, p.partials);
+    if (AMAX_ONLY) {
+        if (RHT && LOGM == 0) amax_bits = __float_as_uint(__uint_as_float(amax_bits) * kRht16Norm);
+        write_partial(amax_bits, p.partials);
+    }
 }
 
 // ------------------------------------- rowwise 1D, stochastic rounding ------
@@ -520,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 uint32_t w = jp == 0 ? v[i].x : jp == 1 ? v[i].y : jp == 2 ? v[i].z : v[i].w;
-                if (RHT && LOGM == 0 && !AMAX_ONLY) {   // signs folded into the unpack (sign words from the parameter bank)
+                if (RHT && LOGM == 0) {   // signs folded into the unpack (sign words from the parameter bank)
                     y[i] = make_float2(bf16_lo_signed(w, p.rht_sign.m[i]), bf16_hi_signed(w, p.rht_sign.m[i]));
                     continue;
                 }
@@ -550,9 +554,13 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
                         y[i] = __fadd2_rn(o, __fmul2_rn(y[i], make_float2(sg, sg)));
                     }
                 }
-                constexpr float c = rht_norm<LOGM>();
+                // The 16-point amax pass leaves out the 1/4 here and applies it
+                // once to the maximum (kRht16Norm).
+                if (!(AMAX_ONLY && LOGM == 0)) {
+                    constexpr float c = rht_norm<LOGM>();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) y[i] = __fmul2_rn(y[i], make_float2(c, c));
+                    for (int i = 0; i < 16; ++i) y[i] = __fmul2_rn(y[i], make_float2(c, c));
+                }
             }
             float bm0 = 0.0f, bm1 = 0.0f;
 #pragma unroll
@@ -634,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, 2) cols_kernel(Params p) {
         __syncthreads();
     }
     if (AMAX_ONLY) {
+        if (RHT && LOGM == 0) amax_bits = __float_as_uint(__uint_as_float(amax_bits) * kRht16Norm);
         write_partial(amax_bits, p.partials);
         if (p.partials2) {
             __syncthreads();   // write_partial's shared scratch is reused

@@ -125,6 +125,20 @@ def test_tiny_and_huge_magnitudes():
     check_1d(_bits(huge), rht=True, rounding=1)
 
 
+def test_rht_subnormal_inputs():
+    """RHT of bf16 subnormals: the butterfly sums and their quarter fall in
+    binary32's subnormal range, where the amax passes' single 1/4 scaling of
+    the maximum must still equal the maximum of the scaled values."""
+    rng = np.random.default_rng(5)
+    tiny = (rng.standard_normal((32, 64)) * 2.0 ** -130).astype(np.float32)
+    tiny[3, 7] = 2.0 ** -133                      # bf16's smallest subnormal
+    tiny[20, 40] = -(2.0 ** -126)
+    x = _bits(tiny)
+    for rounding in (0, 1):
+        check_1d(x, rht=True, rounding=rounding, sr_seed=4)
+        check_1d(x, transpose=True, rht=True, rounding=rounding, sr_seed=4)
+
+
 def test_scale_underflow_blocks():
     vals = np.full((2, 64), 2.0 ** -12, dtype=np.float32)
     vals[0, 0] = 3e4
