@@ -1,12 +1,16 @@
-// quant.cu -- NVFP4 quantizer kernels for sm_100a (HBM-bandwidth bound).
+// quant.cu -- NVFP4 quantizer kernels for sm_100a.  The round-to-nearest
+// passes are bound by HBM bandwidth; the stochastic-rounding and RHT passes
+// by instruction issue (16 Philox bits per element, the butterflies).
 //
 // Steps (sources: "Melatih model dalam 4 bit: pengaman numerik di balik NVFP4",
 // "Anatomi NVFP4" and "Empat pengaman"; "MXFP4 和 NVFP4 的区别", "精度核心:
 // 两级分层缩放", "随机舍入", "随机 Hadamard 变换", "构造 Hadamard 矩阵的方法";
 // "NVFP4 Is a Scaling System, Not Just a 4-Bit Number", "Why two levels":
 // the global scale comes from the tensor amax before the block maxima):
-//   pass 1 (amax):  A = max |Q| over the tensor (Q rotated when RHT is on);
-//                   one partial maximum per CTA into the caller's workspace.
+//   pass 1 (amax):  A = max |Q| over the tensor (Q rotated when RHT is on;
+//                   the 16-point transform's 1/4 is applied to the maximum,
+//                   see kRht16Norm); one partial maximum per CTA into the
+//                   caller's workspace.
 //   pass 2 (encode): every CTA folds the partials into A, s_global =
 //                   RN(A / 2688); per 16-block: block amax, E4M3 scale, E2M1
 //                   codes (RNE or stochastic rounding), packed two per byte.
