@@ -545,6 +545,10 @@ def e2e(torch, N, step, s, args, dist=None, world=1, dev=None):
     # have crossed and the last one's early results overlap its later work.
     need = {0: "x", 1: "w", 3: "dy"}              # op index -> the input it first reads
     done_by = {2: "y", 4: "dx", 5: "dw"}          # op index -> the result it completes
+    names = [o[0] for o in step.ops]
+    assert (names[0].startswith("quantize_dual X") and names[1].startswith("quantize_2d W")
+            and names[2] == "gemm fprop" and names[3].startswith("quantize_dual dY")
+            and names[4] == "gemm dgrad" and names[5] == "gemm wgrad"), names
 
     def one(k):
         b = sets[k % 2]
