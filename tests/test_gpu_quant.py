@@ -182,6 +182,26 @@ def test_quantize_2d(shape):
                                                                      expand_2d=True)) is None
 
 
+def test_quantize_2d_ragged_multi_wave():
+    """More 128 x 256 tiles (21 x 17 = 357) than CTAs, with a 16-row last
+    tile row and a 16-column last tile column: every CTA prefetches a next
+    tile, some of them ragged."""
+    w = G.make_tensor(2576, 4112, seed=580, dist="normal", scale=0.02, outlier_frac=0.001,
+                      outlier_mode="mul", outlier_value=30.0)
+    q = N.quantize_2d(to_device_bf16(w))
+    torch.cuda.synchronize()
+    assert N.nvfp4_get_error() == 0
+    cr, cc, sc, sg = O.quantize_2d(w)
+    R, C = w.shape
+    assert q.global_scale.item() == sg
+    assert first_mismatch(q.scales.cpu().numpy(), sc) is None
+    assert first_mismatch(q.codes.cpu().numpy(), cr) is None
+    assert first_mismatch(q.codes_col.cpu().numpy(), cc) is None
+    assert first_mismatch(q.scales_mma.cpu().numpy(), mma_layout(sc, R, C // 16, expand_2d=True)) is None
+    assert first_mismatch(q.scales_mma_col.cpu().numpy(), mma_layout(np.ascontiguousarray(sc.T), C, R // 16,
+                                                                     expand_2d=True)) is None
+
+
 def test_quantize_2d_tiny_linear_weight():
     _, w = G.tiny_linear()
     q = N.quantize_2d(to_device_bf16(w), columnwise=False)
