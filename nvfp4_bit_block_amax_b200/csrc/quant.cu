@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
     int64_t u = wid * U;
     const int64_t uend = total;
     const int64_t kb = p.cols >> 4;
+    const int64_t chunks512 = p.chunks_k << 9;         // bytes per 128-row band of the GEMM scale layout
     const bool a32 = ((reinterpret_cast<uintptr_t>(p.x) & 31u) == 0) && ((p.ld & 15) == 0);
     uint32_t amax_bits = 0;
     if (u < uend) {
@@ -349,14 +350,18 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(Params p) {
                     *reinterpret_cast<uint2*>(p.codes + rr[k] * (p.cols >> 1) + (cc[k] >> 1)) = make_uint2(lo, hi);
                     if (p.scales) p.scales[rr[k] * kb + b] = (uint8_t)bs.code;
                 }
-                if (p.scales_mma) {
+                if (p.scales_mma && ok[k]) {
                     // Blocks 4g .. 4g+3 of a row are 4 consecutive bytes of the
-                    // GEMM layout: lanes 4g .. 4g+3 gather them into one word.
-                    uint32_t word = bs.code;
-                    word |= __shfl_down_sync(0xFFFFFFFFu, word, 1) << 8;
-                    word |= __shfl_down_sync(0xFFFFFFFFu, word, 2) << 16;
-                    if (ok[k] && (lane & 3) == 0)
-                        *reinterpret_cast<uint32_t*>(p.scales_mma + mma_scale_offset(rr[k], b, p.chunks_k)) = word;
+                    // GEMM layout, so lanes 4g .. 4g+3 each store their own byte
+                    // (the four land in one sector; gathering them into a word
+                    // first cost two shuffles and the full offset arithmetic in
+                    // every lane).  This is mma_scale_offset(r, b) with the row
+                    // part in 32 bits (r < 2^31) and b & 3 = lane & 3.  Bytes of
+                    // a group past the row's end stay as the launch zeroed them.
+                    const uint32_t r32 = (uint32_t)rr[k];
+                    const int64_t off = (int64_t)(r32 >> 7) * chunks512 + ((cc[k] >> 6) << 9) +
+                                        (int64_t)(((r32 & 31u) << 4) | (((r32 >> 5) & 3u) << 2) | (uint32_t)(lane & 3));
+                    p.scales_mma[off] = (uint8_t)bs.code;
                 }
             }
         }
