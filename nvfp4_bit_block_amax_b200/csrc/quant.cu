@@ -399,6 +399,7 @@ __global__ void __launch_bounds__(kThreads) rows_sr_kernel(Params p) {
     const int64_t step_rows = nwarps / spr, step_seg = nwarps - step_rows * spr;
     const bool a32 = ((reinterpret_cast<uintptr_t>(p.x) & 31u) == 0) && ((p.ld & 15) == 0);
     const bool c16 = ((C & 63) == 0) && ((reinterpret_cast<uintptr_t>(p.codes) & 15u) == 0);
+    const int64_t chunks512 = p.chunks_k << 9;         // bytes per 128-row band of the GEMM scale layout
     for (; item < items; item += nwarps) {
         const int64_t col0 = ((seg << 5) + lane) << 6;
         const int nb = col0 < C ? (int)min((int64_t)4, (C - col0) >> 4) : 0;   // blocks of this unit inside the row
@@ -463,8 +464,14 @@ __global__ void __launch_bounds__(kThreads) rows_sr_kernel(Params p) {
                     if (b < nb) sp[b] = (uint8_t)(sword >> (8 * b));
             }
             // blocks 4g .. 4g+3 of the row: one word of the GEMM layout (zeros past the row's end)
-            if (p.scales_mma)
-                *reinterpret_cast<uint32_t*>(p.scales_mma + mma_scale_offset(row, col0 >> 4, p.chunks_k)) = sword;
+            if (p.scales_mma) {
+                // mma_scale_offset(row, col0 / 16) with the row part in 32 bits
+                // (row < 2^31) and col0 / 16 a multiple of 4
+                const uint32_t r32 = (uint32_t)row;
+                const int64_t off = (int64_t)(r32 >> 7) * chunks512 + ((col0 >> 6) << 9) +
+                                    (int64_t)(((r32 & 31u) << 4) | (((r32 >> 5) & 3u) << 2));
+                *reinterpret_cast<uint32_t*>(p.scales_mma + off) = sword;
+            }
         }
         row += step_rows;
         seg += step_seg;
